@@ -1,0 +1,445 @@
+#!/usr/bin/env python
+"""Benchmark of the SVDQuant W4A4 linear layer on B200.
+
+One step = one forward pass of the layer's hot path over one batch:
+svdq_quantize_act (smoothing, NVFP4 quantisation, low-rank down-projection)
+then svdq_linear (block-scaled FP4 GEMM + low-rank up-projection + bias).
+The residual packer runs once per weight; it is timed separately and
+reported beside the step (pack_residual_us).
+
+Default workload: the FLUX.1-shaped attention QKV projection, M = 4608
+tokens (4096 image + 512 text), K = 3072, N = 9216, rank 32, synthetic data.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU runs are independent replicas (the layer is one GPU's work; there
+is no exchange step), launched one process per GPU by torchrun; the value is
+all ranks' work divided by the slowest rank's device time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "SVDQuant W4A4 linear effective TFLOPS & µs/layer; % of B200 FP4/HBM roofline"
+UNIT = "TFLOP/s"
+L2_FLUSH_BYTES = 512 << 20  # > 4x the 126 MB L2
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="flux_qkv")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- peaks ---
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# FP4 dense / bf16 dense on B200: 9 / 2.25 PFLOP/s (spec sheet, dense)
+FP4_OVER_BF16 = 4.0
+
+
+# ---------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), max=float(parts[2]), util=float(parts[4]),
+                                     hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        load = [r for r in rows if r["util"] > 0] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(load)}
+
+
+# ------------------------------------------------------------- workload ---
+
+def workload_desc(name, M, K, N, r):
+    return {"workload": f"{name}: M={M} K={K} N={N} rank={r}, NVFP4 group 16",
+            "M": M, "K": K, "N": N, "rank": r, "l2": "flushed (512 MB write) before every step"}
+
+
+def setup_layer(name: str, device):
+    import torch
+    import bit_w4a4_quantized_smooth_b200 as svdq
+    from bit_w4a4_quantized_smooth_b200 import prep
+    from svdq_inputs import make_layer_inputs
+
+    li = make_layer_inputs(name)
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+
+    X = bf16(li.X)
+    W = bf16(li.W)
+    bias = None if li.bias is None else bf16(li.bias)
+    lam, inv = prep.smoothing(X, W)
+    L1, L2, R = prep.lowrank(W, lam, li.r)
+    del W
+    rc, rs = svdq.pack_residual(R)
+    torch.cuda.synchronize()
+    return dict(li=li, X=X, inv=inv, L1=L1, L2=L2, R=R, bias=bias, rc=rc, rs=rs,
+                M=li.M, K=li.K, N=li.N, r=li.r)
+
+
+def layer_flops(M, K, N, r):
+    return 2.0 * M * N * K + 2.0 * M * (K + N) * r
+
+
+def linear_bytes(M, K, N, r):
+    """Algorithmic bytes of the layer: X bf16, packed R, L1, L2, Y, bias."""
+    return 2 * M * K + N * K // 2 + N * K // 16 + 2 * K * r + 2 * r * N + 2 * M * N + 2 * N
+
+
+# -------------------------------------------------------- oracle (CPU) ---
+
+def oracle_sample(X_bits, inv, L1_bits, L2_bits, R, bias_bits, M, K, N, r, target_s):
+    """Time the oracle's forward (activation step + linear) on a bounded row
+    sample; returns (TFLOP/s, rows, seconds, threads)."""
+    import oracle
+    rc, rs = oracle.pack_residual(R)  # per-weight preparation, not timed
+
+    def run(rows):
+        t0 = time.perf_counter()
+        xc, xs, T = oracle.quantize_act(X_bits[:rows], inv, L1_bits, r)
+        oracle.linear_rows(xc, xs, T, rc, rs, L2_bits, bias_bits, rows, K, N, r, np.arange(rows))
+        return time.perf_counter() - t0
+
+    rows = 4
+    t = run(rows)
+    rows = int(max(4, min(M, rows * target_s / max(t, 1e-3))))
+    t = run(rows)
+    return layer_flops(rows, K, N, r) / t / 1e12, rows, t, oracle.num_threads()
+
+
+# ------------------------------------------------------------- our arm ---
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import bit_w4a4_quantized_smooth_b200 as svdq
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    L = setup_layer(args.workload, device)
+    M, K, N, r = L["M"], L["K"], L["N"], L["r"]
+    X, inv, L1, L2, bias, rc, rs = L["X"], L["inv"], L["L1"], L["L2"], L["bias"], L["rc"], L["rs"]
+    cb, sb = svdq.packed_sizes(M, K)
+    xc = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+    xs = torch.empty(sb, dtype=torch.uint8, device=device)
+    T = torch.empty((M, r), dtype=torch.bfloat16, device=device) if r else None
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        svdq.quantize_act(X, inv, L1, x_codes=xc, x_scales=xs, T=T, stream=stream)
+        svdq.linear(xc, xs, T, rc, rs, L2, bias, M, K, N, Y=Y, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st, where = svdq.sync_status()
+    if st != 0:
+        raise RuntimeError(f"kernel wait expired during warm-up (id {where})")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(args.steps):
+        flush.zero_()
+        e0, e1, e2 = ev[i]
+        e0.record(stream)
+        svdq.quantize_act(X, inv, L1, x_codes=xc, x_scales=xs, T=T, stream=stream)
+        e1.record(stream)
+        svdq.linear(xc, xs, T, rc, rs, L2, bias, M, K, N, Y=Y, stream=stream)
+        e2.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    qa_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    lin_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    step_ms = [a + b for a, b in zip(qa_ms, lin_ms)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    st, where = svdq.sync_status()
+    if st != 0:
+        raise RuntimeError(f"kernel wait expired in the timed region (id {where})")
+
+    flops = layer_flops(M, K, N, r)
+    ms_per_step = total_ms / args.steps
+    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+
+    # ---- per-kernel figures (this rank) ----
+    qa_us = 1e3 * statistics.mean(qa_ms)
+    lin_us = 1e3 * statistics.mean(lin_ms)
+
+    # plain FP4 GEMM (rank 0 branch switched off) on the same operands, for
+    # the low-rank overhead
+    def time_linear(rr, reps=20):
+        es = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)]
+        for a, b in es:
+            flush.zero_()
+            a.record(stream)
+            svdq.linear(xc, xs, T if rr else None, rc, rs, L2 if rr else None, bias, M, K, N, Y=Y,
+                        stream=stream)
+            b.record(stream)
+        torch.cuda.synchronize()
+        return 1e3 * statistics.mean(a.elapsed_time(b) for a, b in es)
+
+    lin_r0_us = time_linear(0) if r else lin_us
+
+    # residual packer, once per weight
+    pk = []
+    for _ in range(10):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        svdq.pack_residual(L["R"], r_codes=rc, r_scales=rs, stream=stream)
+        b.record(stream)
+        pk.append((a, b))
+    torch.cuda.synchronize()
+    pack_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in pk)
+
+    # ---- end to end through the public API with host buffers ----
+    X_host = torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True)
+    X_host.copy_(X)
+    Y_host = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+    X_dev = torch.empty_like(X)
+    e2e = []
+    for i in range(max(3, args.warmup) + args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        X_dev.copy_(X_host, non_blocking=True)
+        svdq.quantize_act(X_dev, inv, L1, x_codes=xc, x_scales=xs, T=T, stream=stream)
+        svdq.linear(xc, xs, T, rc, rs, L2, bias, M, K, N, Y=Y, stream=stream)
+        Y_host.copy_(Y, non_blocking=True)
+        b.record(stream)
+        if i >= max(3, args.warmup):
+            e2e.append((a, b))
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * flops * len(e2e) / (e2e_ms * 1e-3) / 1e12
+
+    peaks = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    achieved = flops / (lin_us * 1e-6) / 1e12
+    qa_bytes = 2 * M * K + M * K // 2 + M * K // 16 + 2 * M * r + 2 * K * r + 4 * K
+    layer_roof_us = max(flops / (fp4_peak * 1e12), linear_bytes(M, K, N, r) / (peaks["hbm_gbs"] * 1e9)) * 1e6
+
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4",
+        "data": "synthetic",
+        "config": dict(workload_desc(args.workload, M, K, N, r), parallelism=f"replicas{world}"),
+        "us_per_layer": round(1e3 * ms_per_step, 2),
+        "quantize_act_us": round(qa_us, 2),
+        "linear_us": round(lin_us, 2),
+        "linear_r0_us": round(lin_r0_us, 2),
+        "lowrank_overhead": round(lin_us / lin_r0_us - 1.0, 4),
+        "pack_residual_us": round(pack_us, 2),
+        "pack_residual_gbs": round((K * N * 4 + N * K // 2 + N * K // 16) / (pack_us * 1e-6) / 1e9, 1),
+        "quantize_act_gbs": round(qa_bytes / (qa_us * 1e-6) / 1e9, 1),
+        "layer_roofline_us": round(layer_roof_us, 2),
+        "layer_roofline_frac": round(layer_roof_us / (1e3 * ms_per_step), 4),
+        "roofline": {
+            "kernel": "linear_kernel",
+            "bound": "tensor",
+            "achieved": round(achieved, 1),
+            "peak": round(fp4_peak, 1),
+            "unit": "TFLOP/s",
+            "frac": round(achieved / fp4_peak, 4),
+            "traffic": None,
+            "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 4 (FP4/bf16 dense ratio)",
+        },
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
+                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+    }
+    return out, L
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        out, L = run_ours(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            li = L["li"]
+            to_np = lambda t: None if t is None else t.detach().cpu().contiguous()
+            bits = lambda t: None if t is None else to_np(t).view(torch.int16).numpy().view(np.uint16)
+            v, rows, secs, thr = oracle_sample(li.X, to_np(L["inv"]).numpy(), bits(L["L1"]),
+                                               bits(L["L2"]), to_np(L["R"]).numpy(), li.bias,
+                                               L["M"], L["K"], L["N"], L["r"], args.cpu_seconds)
+            out["cpu_baseline"] = {"value": round(v, 6), "unit": UNIT, "cores": thr, "kind": "oracle",
+                                   "sample": f"{rows} of {L['M']} rows (activation step + linear), "
+                                             f"{secs:.1f} s, fp64 OpenMP"}
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    return 0
+
+
+def run_reference(args):
+    """The oracle (plain CPU implementation) on the same workload and metric."""
+    import oracle
+    from svdq_inputs import make_layer_inputs
+    li = make_layer_inputs(args.workload)
+    lam, inv = oracle.smooth(li.Xcal, li.W)
+    L1, L2, R, _ = oracle.lowrank(li.W, lam, li.r)
+    rc, rs = oracle.pack_residual(R)
+    M, K, N, r = li.M, li.K, li.N, li.r
+    per_step_s = max(0.5, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    # rows per step sized from one probe
+    t0 = time.perf_counter()
+    xc, xs, T = oracle.quantize_act(li.X[:4], inv, L1 if r else None, r)
+    oracle.linear_rows(xc, xs, T, rc, rs, L2 if r else None, li.bias, 4, K, N, r, np.arange(4))
+    probe = time.perf_counter() - t0
+    rows = int(max(1, min(M, 4 * per_step_s / max(probe, 1e-3))))
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        xc, xs, T = oracle.quantize_act(li.X[:rows], inv, L1 if r else None, r)
+        oracle.linear_rows(xc, xs, T, rc, rs, L2 if r else None, li.bias, rows, K, N, r, np.arange(rows))
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = layer_flops(rows, K, N, r) * len(times) / total / 1e12
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 6),
+        "unit": UNIT,
+        "n_gpus": args.gpus,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / len(times), 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": dict(workload_desc(args.workload, M, K, N, r), parallelism="cpu"),
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": f"{rows} of {M} rows per step"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,51 @@
+"""Offline preparation of one layer on the GPU (run once per weight, untimed).
+
+SVDQuant's preparation (chattools.cn article 584, "technical principles";
+ai-digest.ru abstract): smoothing factors move activation outliers into the
+weights, the SVD of the smoothed weight gives the 16-bit low-rank branch,
+and the rest is the residual that the packer quantises to 4 bits.
+
+    lambda_j = sqrt(max_i |X_ij|) / sqrt(max_n |W_jn|)   (1 if either max is 0)
+    Wh = diag(lambda) W,  Wh ~ U_r S_r V_r^T  (top-r eigenpairs of the Gram matrix)
+    L1 = bf16(U_r S_r), L2 = bf16(V_r^T), R = fp32(Wh - L1 L2)
+
+It uses torch's library linear algebra (matmul, eigh) in fp64 on the device:
+preparation is not part of the forward pass that the library's kernels run.
+"""
+
+from __future__ import annotations
+
+import torch
+
+
+def smoothing(Xcal: torch.Tensor, W: torch.Tensor):
+    """-> (lambda fp32 [K], inv_lambda fp32 [K])."""
+    a = Xcal.abs().amax(dim=0).double()
+    b = W.abs().amax(dim=1).double()
+    lam = torch.where((a == 0) | (b == 0), torch.ones_like(a), a.sqrt() / b.sqrt()).float()
+    inv = torch.ones_like(lam) / lam  # fp32 quotient, rounded once
+    return lam, inv
+
+
+def lowrank(W: torch.Tensor, lam: torch.Tensor, r: int):
+    """-> (L1 bf16 [K][r] or None, L2 bf16 [r][N] or None, R fp32 [K][N])."""
+    Wh = lam.double()[:, None] * W.double()
+    K, N = Wh.shape
+    if r == 0:
+        return None, None, Wh.float()
+    if K <= N:
+        G = Wh @ Wh.T
+        w, Q = torch.linalg.eigh(G)
+        U = Q[:, -r:].flip(1)
+        s = w[-r:].flip(0).clamp_min(0).sqrt()
+        V = (Wh.T @ U) / torch.where(s > 0, s, torch.ones_like(s))
+    else:
+        G = Wh.T @ Wh
+        w, Q = torch.linalg.eigh(G)
+        V = Q[:, -r:].flip(1)
+        s = w[-r:].flip(0).clamp_min(0).sqrt()
+        U = (Wh @ V) / torch.where(s > 0, s, torch.ones_like(s))
+    L1 = (U * s).to(torch.bfloat16)
+    L2 = V.T.contiguous().to(torch.bfloat16)
+    R = (Wh - L1.double() @ L2.double()).float()
+    return L1.contiguous(), L2.contiguous(), R.contiguous()

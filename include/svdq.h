@@ -1,0 +1,144 @@
+/*
+ * svdq.h -- C ABI of the SVDQuant W4A4 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer (SVDQuant, "Absorbing outliers by low-rank components for 4-bit
+ * diffusion models"; abstract as translated on ai-digest.ru, and the
+ * "technical principles" section of chattools.cn article 584):
+ *
+ *     Y = Xh L1 L2 + Q(Xh) Q(R) + bias,      Xh = X diag(lambda)^-1
+ *
+ * X [M][K] is the activation, lambda [K] the smoothing factors that move
+ * activation outliers into the weights, L1 [K][r] and L2 [r][N] the 16-bit
+ * low-rank branch from the SVD of diag(lambda) W, R = diag(lambda) W - L1 L2
+ * the residual, and Q() the 4-bit NVFP4 quantiser: E2M1 values with one
+ * unsigned E4M3 scale per 16 consecutive elements along K, scale = amax / 6.
+ * The pages' engine fuses the low-rank branch into the 4-bit kernels to avoid
+ * a second pass over the activation (ai-digest.ru abstract, chattools.cn
+ * "kernel fusion" bullet); here the down-projection Xh L1 shares the
+ * quantiser's read of X and the up-projection (Xh L1) L2 accumulates into
+ * the 4-bit GEMM's tensor-memory accumulator.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All tensors are dense, row-major, in DEVICE memory, allocated and owned
+ *    by the caller.  The library allocates no memory and keeps no state
+ *    besides a per-device status word (see svdq_sync_status).
+ *  - bf16 tensors are passed as `const void*` / `void*` (IEEE bfloat16).
+ *  - Every pointer must be 16-byte aligned.  K must be a multiple of 64,
+ *    N a multiple of 16, r one of 0, 16, 32, ..., 128, M >= 1.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *    are asynchronous and stream-ordered; none synchronises.
+ *  - Argument errors are detected on the host before anything is launched
+ *    and returned as a status; no call aborts or exits.
+ *  - Inputs must be finite; NaN or Inf gives unspecified codes.
+ *
+ * Packed NVFP4 layout (codes and scales)
+ * --------------------------------------
+ *  - codes: uint8 [rows][K/2]; element k of a row is in byte k/2, in the
+ *    low nibble for even k and the high nibble for odd k.  E2M1 code: bit 3
+ *    sign, bits 0-2 magnitude index into {0, .5, 1, 1.5, 2, 3, 4, 6}.
+ *  - scales: uint8 unsigned-E4M3, one per 16 elements along K, in the
+ *    tensor cores' block-scale tile layout: rows are padded to a multiple of
+ *    128; tile (row/128, g/4) (g = k/16) is 512 contiguous bytes, tiles of a
+ *    128-row band are consecutive along K, and inside a tile (row, g) is at
+ *    byte (row % 32) * 16 + ((row % 128) / 32) * 4 + (g % 4).  Scales of the
+ *    padding rows are written as 0.
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,       /* null pointer, negative size */
+  SVDQ_ERR_UNSUPPORTED_SHAPE = 2, /* K % 64, N % 16, r not in {0,16,...,128} */
+  SVDQ_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned */
+  SVDQ_ERR_CUDA = 4,              /* a CUDA runtime/driver call failed */
+  SVDQ_ERR_TIMEOUT = 5            /* a kernel's bounded wait expired */
+} svdq_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* svdq_status_string(int status);
+
+/* Bytes of the packed buffers for `rows` vectors of length K:
+ * codes_bytes = rows * K / 2, scales_bytes = ceil(rows / 128) * 128 * K / 16.
+ * Host-only; K must be a multiple of 64. */
+int svdq_packed_sizes(int64_t rows, int64_t K, size_t* codes_bytes, size_t* scales_bytes);
+
+/*
+ * Residual packer, run once per weight (the 4-bit residual of the SVDQuant
+ * principles: the part of diag(lambda) W left after removing the low-rank
+ * branch is quantised to 4 bits).
+ *   R        fp32 [K][N]   residual diag(lambda) W - L1 L2
+ *   r_codes  uint8 [N][K/2]        output: NVFP4 codes, one row per output
+ *                                   channel n, groups of 16 along K
+ *   r_scales uint8, svdq_packed_sizes(N, K) bytes, tile layout above
+ */
+int svdq_pack_residual(const float* R, int64_t K, int64_t N, uint8_t* r_codes,
+                       uint8_t* r_scales, void* stream);
+
+/*
+ * Activation step of one forward pass: smoothing, 4-bit quantisation and the
+ * low-rank down-projection from one read of X.
+ *   X          bf16 [M][K]
+ *   inv_lambda fp32 [K]     1 / lambda_j, rounded to fp32 by the caller;
+ *                           Xh = RN_f32(X * inv_lambda) element-wise
+ *   L1         bf16 [K][r]  low-rank down-projection (NULL iff r == 0)
+ *   x_codes    uint8 [M][K/2]               output: NVFP4 codes of Xh
+ *   x_scales   uint8, svdq_packed_sizes(M, K) output: scales of Xh
+ *   T          bf16 [M][r]  output: bf16(bf16(Xh) L1), fp32 accumulation
+ *                           (NULL iff r == 0)
+ * NVFP4 group rule (16 values v along K): s = E4M3_RNE_satfinite(
+ * RN_f32(amax / 6)); rcp = RN_f32(1 / decode(s)) (0 if decode(s) == 0);
+ * q_i = E2M1_RNE_satfinite(RN_f32(v_i * rcp)).
+ */
+int svdq_quantize_act(const void* X, const float* inv_lambda, const void* L1, int64_t M,
+                      int64_t K, int64_t r, uint8_t* x_codes, uint8_t* x_scales, void* T,
+                      void* stream);
+
+/*
+ * Fused 4-bit linear: Y = deq(x) deq(R)^T + T L2 + bias, written as bf16.
+ * The block-scaled FP4 product and the rank-r bf16 product accumulate in
+ * the same fp32 tensor-memory accumulator; bias is added in fp32 and the
+ * result rounded once to bf16.
+ *   x_codes, x_scales   from svdq_quantize_act (M rows)
+ *   T                   bf16 [M][r] (NULL iff r == 0)
+ *   r_codes, r_scales   from svdq_pack_residual (N rows)
+ *   L2                  bf16 [r][N] (NULL iff r == 0)
+ *   bias                bf16 [N] or NULL
+ *   Y                   bf16 [M][N] output
+ */
+int svdq_linear(const uint8_t* x_codes, const uint8_t* x_scales, const void* T,
+                const uint8_t* r_codes, const uint8_t* r_scales, const void* L2,
+                const void* bias, int64_t M, int64_t K, int64_t N, int64_t r, void* Y,
+                void* stream);
+
+/*
+ * Failure detection.  Every wait inside the kernels is bounded (default
+ * 2 s, or SVDQ_WAIT_TIMEOUT_MS from the environment at first use); a wait
+ * that expires records SVDQ_ERR_TIMEOUT in the current device's status word
+ * and the kernel returns without hanging the GPU.
+ *
+ * svdq_sync_status synchronises `stream`, returns the recorded status of
+ * the current device (SVDQ_OK if none; SVDQ_ERR_CUDA if the stream reports
+ * an error) and clears it.  `where`, if not NULL, receives the id of the
+ * wait that expired (0 if none).
+ */
+int svdq_sync_status(void* stream, int* where);
+
+/* Self test of the bounded wait: launches one CTA that waits on a barrier
+ * nothing will complete, with the given limit in nanoseconds; the wait
+ * expires and records SVDQ_ERR_TIMEOUT, read back with svdq_sync_status. */
+int svdq_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H_ */

@@ -1,0 +1,94 @@
+"""The C-ABI library loads, exports every symbol the header declares, and
+rejects bad arguments on the host before touching a GPU (no compute call is
+made here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "svdq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bit_w4a4_quantized_smooth_b200 import build, binding
+    build.build()
+    return binding.load()
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(svdq_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert {"svdq_pack_residual", "svdq_quantize_act", "svdq_linear"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    from bit_w4a4_quantized_smooth_b200 import status_string
+    assert status_string(0) == "SVDQ_OK"
+    assert status_string(5) == "SVDQ_ERR_TIMEOUT"
+    assert status_string(99) == "SVDQ_UNKNOWN_STATUS"
+
+
+def test_packed_sizes(lib):
+    from bit_w4a4_quantized_smooth_b200 import packed_sizes, SvdqError
+    assert packed_sizes(4608, 3072) == (4608 * 1536, 4608 * 192)
+    assert packed_sizes(1, 64) == (32, 128 * 4)
+    assert packed_sizes(200, 320) == (200 * 160, 256 * 20)
+    with pytest.raises(SvdqError):
+        packed_sizes(10, 100)
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def test_linear_validation(lib):
+    P = ctypes.c_void_p
+    ok = dict(xc=FAKE, xs=FAKE, T=FAKE, rc=FAKE, rs=FAKE, L2=FAKE, bias=None, M=128, K=256, N=256,
+              r=32, Y=FAKE)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return lib.svdq_linear(P(a["xc"]), P(a["xs"]), P(a["T"]), P(a["rc"]), P(a["rs"]), P(a["L2"]),
+                               P(a["bias"]), a["M"], a["K"], a["N"], a["r"], P(a["Y"]), None)
+
+    assert call(xc=None) == 1
+    assert call(Y=None) == 1
+    assert call(T=None) == 1           # r > 0 needs T
+    assert call(M=0) == 1
+    assert call(K=100) == 2
+    assert call(N=24) == 2
+    assert call(r=24) == 2
+    assert call(r=144) == 2
+    assert call(xc=FAKE + 8) == 3
+    assert call(bias=FAKE + 2) == 3
+
+
+def test_quantize_and_pack_validation(lib):
+    P = ctypes.c_void_p
+    q = lib.svdq_quantize_act
+    assert q(P(FAKE), P(FAKE), P(FAKE), 16, 64, 16, P(FAKE), P(FAKE), None, None) == 1  # T missing
+    assert q(P(FAKE), P(FAKE), None, 16, 96, 0, P(FAKE), P(FAKE), None, None) == 2
+    assert q(P(FAKE + 4), P(FAKE), None, 16, 64, 0, P(FAKE), P(FAKE), None, None) == 3
+    p = lib.svdq_pack_residual
+    assert p(None, 64, 16, P(FAKE), P(FAKE), None) == 1
+    assert p(P(FAKE), 64, 8, P(FAKE), P(FAKE), None) == 2
+    assert p(P(FAKE), 64, 16, P(FAKE + 1), P(FAKE), None) == 3
+    assert lib.svdq_selftest_wait_timeout(0, None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    from bit_w4a4_quantized_smooth_b200 import binding
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "_LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        binding.load()

@@ -1,0 +1,162 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+* packed codes and scales: bit-exact (integer work decided in fp32 on both
+  sides: the same RN_f32 products and quotients, then RNE to E4M3/E2M1);
+* T = bf16(bf16(Xh) L1): within one bf16 ulp of the oracle's fp64 sum
+  rounded once (fp32 tensor-core accumulation may flip a rounding), and at
+  least 98 % of the elements bit-identical;
+* Y: relative Frobenius error <= 2e-3 against the oracle's fp64 Y, where
+  the output rounding to bf16 alone contributes about 1e-3.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from tests._cases import bf16_bits_to_f64, bf16_to_np_bits, prepare, to_device
+
+pytestmark = pytest.mark.gpu
+
+Y_TOL = 2e-3
+
+# (workload, M, K, N, r): several tiles, ragged M / N / K tails, r = 0,
+# r = 128 (two low-rank stages), M = 1, an 8-CTA cluster (K = 2048)
+SMALL = [
+    ("tiny", None, None, None, None),            # the full tiny layer 256 x 1024 x 1024, r 16
+    ("flux_qkv", 200, 320, 272, 32),             # ragged M, N (one 128-row scale band) and K
+    ("flux_mlp_up", 130, 256, 512, 0),           # no low-rank branch
+    ("flux_mlp_down", 384, 512, 256, 128),       # GELU inputs, two low-rank stages
+    ("flux_qkv", 1, 1024, 256, 64),              # one token
+    ("sweep_3072", 128, 2048, 256, 48),          # cluster of 8 along K, r = 48
+    ("flux_qkv", 300, 192, 528, 16),             # K = 3 chunks, N tail of 16 columns
+]
+
+
+def _ids(c):
+    return "-".join(str(x) for x in c)
+
+
+def _torch():
+    import torch
+    assert torch.cuda.is_available()
+    return torch
+
+
+def _lib():
+    import bit_w4a4_quantized_smooth_b200 as svdq
+    svdq.load()
+    return svdq
+
+
+def check_T(T_gpu_bits, T_or_bits):
+    a = bf16_bits_to_f64(T_gpu_bits)
+    b = bf16_bits_to_f64(T_or_bits)
+    same = np.mean(T_gpu_bits == T_or_bits)
+    ulp = np.spacing(np.abs(b).astype(np.float32)).astype(np.float64) * 65536.0  # bf16 ulp
+    tiny = 1e-30 + 1e-6 * np.abs(b).max()
+    assert np.all(np.abs(a - b) <= ulp + tiny), np.abs(a - b).max()
+    assert same >= 0.98, same
+
+
+def rel_fro(Y, ref):
+    return float(np.linalg.norm(Y - ref) / np.linalg.norm(ref))
+
+
+@pytest.mark.parametrize("case", SMALL, ids=_ids)
+def test_pack_residual_bit_exact(case):
+    torch = _torch()
+    svdq = _lib()
+    p = prepare(*case)
+    d = to_device(p)
+    rc, rs = svdq.pack_residual(d["R"])
+    torch.cuda.synchronize()
+    orc, ors = oracle.pack_residual(p.R)
+    assert np.array_equal(rc.cpu().numpy(), orc)
+    assert np.array_equal(rs.cpu().numpy(), ors)
+
+
+@pytest.mark.parametrize("case", SMALL, ids=_ids)
+def test_quantize_act(case):
+    torch = _torch()
+    svdq = _lib()
+    p = prepare(*case)
+    d = to_device(p)
+    xc, xs, T = svdq.quantize_act(d["X"], d["inv"], d["L1"])
+    torch.cuda.synchronize()
+    oxc, oxs, oT = oracle.quantize_act(p.X, p.inv, p.L1, p.r)
+    assert np.array_equal(xc.cpu().numpy(), oxc)
+    assert np.array_equal(xs.cpu().numpy(), oxs)
+    if p.r:
+        check_T(bf16_to_np_bits(T), oT)
+    assert svdq.sync_status()[0] == 0
+
+
+@pytest.mark.parametrize("case", SMALL, ids=_ids)
+def test_linear_on_oracle_operands(case):
+    """The GEMM alone: the oracle's packed operands in, Y compared."""
+    torch = _torch()
+    svdq = _lib()
+    p = prepare(*case)
+    d = to_device(p)
+    oxc, oxs, oT = oracle.quantize_act(p.X, p.inv, p.L1, p.r)
+    orc, ors = oracle.pack_residual(p.R)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    Tt = None if oT is None else dev(oT.view(np.int16)).view(torch.bfloat16)
+    Y = svdq.linear(dev(oxc), dev(oxs), Tt, dev(orc), dev(ors), d["L2"], d["bias"], p.M, p.K, p.N)
+    torch.cuda.synchronize()
+    Yg = bf16_bits_to_f64(bf16_to_np_bits(Y))
+    ref = oracle.linear_rows(oxc, oxs, oT, orc, ors, p.L2, p.bias, p.M, p.K, p.N, p.r, np.arange(p.M))
+    err = rel_fro(Yg, ref)
+    assert err <= Y_TOL, err
+    assert svdq.sync_status()[0] == 0
+
+
+@pytest.mark.parametrize("case", SMALL, ids=_ids)
+def test_layer_end_to_end(case):
+    """quantize_act + linear on the GPU vs the oracle's Y; also the
+    quantisation error against the unquantised X W (reported)."""
+    torch = _torch()
+    svdq = _lib()
+    p = prepare(*case)
+    d = to_device(p)
+    rc, rs = svdq.pack_residual(d["R"])
+    xc, xs, T = svdq.quantize_act(d["X"], d["inv"], d["L1"])
+    Y = svdq.linear(xc, xs, T, rc, rs, d["L2"], d["bias"], p.M, p.K, p.N)
+    torch.cuda.synchronize()
+    Yg = bf16_bits_to_f64(bf16_to_np_bits(Y))
+    oxc, oxs, oT = oracle.quantize_act(p.X, p.inv, p.L1, p.r)
+    orc, ors = oracle.pack_residual(p.R)
+    ref = oracle.linear_rows(oxc, oxs, oT, orc, ors, p.L2, p.bias, p.M, p.K, p.N, p.r, np.arange(p.M))
+    err = rel_fro(Yg, ref)
+    assert err <= Y_TOL, err
+    assert svdq.sync_status()[0] == 0
+
+
+def test_back_to_back_calls_reuse_outputs():
+    """Same buffers, two calls in a row: identical results (no stale state)."""
+    torch = _torch()
+    svdq = _lib()
+    p = prepare("flux_qkv", 200, 320, 272, 32)
+    d = to_device(p)
+    rc, rs = svdq.pack_residual(d["R"])
+    xc, xs, T = svdq.quantize_act(d["X"], d["inv"], d["L1"])
+    Y1 = svdq.linear(xc, xs, T, rc, rs, d["L2"], d["bias"], p.M, p.K, p.N).clone()
+    xs.fill_(0x7F)
+    xc2, xs2, T2 = svdq.quantize_act(d["X"], d["inv"], d["L1"], x_codes=xc, x_scales=xs, T=T)
+    Y2 = svdq.linear(xc2, xs2, T2, rc, rs, d["L2"], d["bias"], p.M, p.K, p.N)
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2)
+
+
+def test_wait_timeout_is_reported():
+    """A bounded wait that expires records SVDQ_ERR_TIMEOUT; the context
+    stays usable afterwards."""
+    torch = _torch()
+    svdq = _lib()
+    assert svdq.sync_status()[0] == 0
+    svdq.selftest_wait_timeout(2_000_000)  # 2 ms
+    st, where = svdq.sync_status()
+    assert st == 5 and where == 1
+    assert svdq.sync_status()[0] == 0  # cleared
+    x = torch.ones(4, device="cuda")
+    assert float(x.sum()) == 4.0
