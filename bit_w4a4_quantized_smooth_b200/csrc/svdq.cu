@@ -15,8 +15,6 @@
 
 namespace {
 
-using svdq::kLinStageBytes;
-using svdq::kLinStages;
 using svdq::kQaStages;
 
 uint64_t g_timeout_ns = 0;
@@ -67,6 +65,20 @@ int make_tmap(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t rank, const 
 }
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA; }
+
+// Streaming multiprocessors of the current device (cached per device id).
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
 
 // Largest cluster size (1, 2, 4, 8) dividing the number of 64-column chunks
 // such that row tiles x cluster stays within about two waves of 148 SMs.
@@ -158,8 +170,8 @@ int svdq_quantize_act(const void* X, const float* inv_lambda, const void* L1, in
   p.cpc = static_cast<int>(K / 64 / ks);
   p.timeout_ns = wait_timeout_ns();
 
-  const size_t stage = 16384 + static_cast<size_t>(r) * 128;
-  const size_t smem = 1024 + kQaStages * stage + (2 * kQaStages + 1) * 8 + 16;
+  const size_t smem = 1024 + kQaStages * static_cast<size_t>(svdq::qa_stage_bytes(static_cast<int>(r))) +
+                      (3 * kQaStages + 1) * 8 + 16;
   if (cudaFuncSetAttribute(svdq::quantize_act_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return SVDQ_ERR_CUDA;
@@ -238,13 +250,16 @@ int svdq_linear(const uint8_t* x_codes, const uint8_t* x_scales, const void* T, 
   p.N = static_cast<int>(N);
   p.r = static_cast<int>(r);
   p.timeout_ns = wait_timeout_ns();
+  p.m_tiles = static_cast<int>((M + svdq::kLinBM - 1) / svdq::kLinBM);
+  p.tiles = p.m_tiles * static_cast<int>((N + svdq::kLinBN - 1) / svdq::kLinBN);
 
-  const size_t smem = 1024 + kLinStages * static_cast<size_t>(kLinStageBytes) + (2 * kLinStages + 1) * 8 + 16;
+  const size_t smem = 1024 + svdq::kLinBarOffset + 16 * 8 + 16;
   if (cudaFuncSetAttribute(svdq::linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return SVDQ_ERR_CUDA;
-  dim3 grid(static_cast<unsigned>((N + svdq::kLinBN - 1) / svdq::kLinBN),
-            static_cast<unsigned>((M + svdq::kLinBM - 1) / svdq::kLinBM));
+  const int sms = sm_count();
+  if (sms <= 0) return SVDQ_ERR_CUDA;
+  dim3 grid(static_cast<unsigned>(p.tiles < sms ? p.tiles : sms));
   svdq::linear_kernel<<<grid, svdq::kLinThreads, smem, static_cast<cudaStream_t>(stream)>>>(
       tm_xc, tm_rc, tm_t, tm_l2, p);
   return launch_status();
