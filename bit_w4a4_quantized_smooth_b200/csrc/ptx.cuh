@@ -179,6 +179,20 @@ __device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t 
                : "memory");
 }
 
+// 32 lanes x 32 bit, 16 consecutive columns: thread t writes lane (base + t).
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -225,6 +239,263 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uin
   d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm100
   d |= static_cast<uint64_t>(layout & 7) << 61;
   return d;
+}
+
+// ----------------------------------------------------- CTA-pair (2-SM) --
+// TMA load into this CTA's shared memory whose completion bytes go to the
+// mbarrier at `bar_cluster` (a shared::cluster address, possibly the peer's).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, uint32_t bar_cluster,
+                                                 int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(tmap), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// MMAs across the CTA pair (issued by the even CTA): A rows split by CTA,
+// B columns split by CTA, D rows in each CTA's own tensor memory.
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Arrive once on the mbarrier at the same shared-memory offset in both CTAs
+// of the pair when all prior tcgen05 ops of this thread are complete.
+__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
+}
+
+// Arrive on an mbarrier given by its shared::cluster address (release at
+// cluster scope: prior writes of this thread are visible to the waiter).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait (acquire at cluster scope) for barriers that threads of the
+// peer CTA arrive on.
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
+                                                  unsigned int where) {
+#pragma unroll 1
+  for (int i = 0; i < 32; ++i)
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+#pragma unroll 1
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      record_timeout(where);
+      return false;
+    }
+  }
+}
+
+// 32 lanes x 32 bit, 8 consecutive columns.
+__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+      : "memory");
+}
+
+// ------------------------------------------------- warp-wide issue (elect) --
+// Issue loops run with the whole warp converged and let elect.sync pick the
+// single lane that executes the instruction: this keeps the loop's values on
+// the warp-uniform path (a loop run by one lane inside a divergent branch
+// issues tcgen05 MMAs at well under half their rate).
+#define SVDQ_ELECT_BEGIN "{\n\t.reg .pred e;\n\t.reg .b32 rx;\n\telect.sync rx|e, 0xffffffff;\n\t"
+#define SVDQ_ELECT_END "\n\t}"
+
+__device__ __forceinline__ void e_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile(SVDQ_ELECT_BEGIN "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" SVDQ_ELECT_END ::"r"(bar),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void e_arrive(uint32_t bar) {
+  asm volatile(SVDQ_ELECT_BEGIN "@e mbarrier.arrive.shared::cta.b64 _, [%0];" SVDQ_ELECT_END ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void e_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile(SVDQ_ELECT_BEGIN "@e mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" SVDQ_ELECT_END ::"r"(
+                   bar_cluster)
+               : "memory");
+}
+
+__device__ __forceinline__ void e_tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int x, int y) {
+  asm volatile(SVDQ_ELECT_BEGIN
+               "@e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+               " [%0], [%1, {%2, %3}], [%4];" SVDQ_ELECT_END ::"r"(dst),
+               "l"(tmap), "r"(x), "r"(y), "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void e_tma_load_3d(uint32_t dst, const void* tmap, uint32_t bar, int x, int y, int z) {
+  asm volatile(SVDQ_ELECT_BEGIN
+               "@e cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+               " [%0], [%1, {%2, %3, %4}], [%5];" SVDQ_ELECT_END ::"r"(dst),
+               "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void e_tma_load_2d_pair(uint32_t dst, const void* tmap, uint32_t bar_cluster, int x,
+                                                   int y) {
+  asm volatile(SVDQ_ELECT_BEGIN
+               "@e cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+               " [%0], [%1, {%2, %3}], [%4];" SVDQ_ELECT_END ::"r"(dst),
+               "l"(tmap), "r"(x), "r"(y), "r"(bar_cluster)
+               : "memory");
+}
+
+__device__ __forceinline__ void e_bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(SVDQ_ELECT_BEGIN
+               "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" SVDQ_ELECT_END ::
+                   "r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void e_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(SVDQ_ELECT_BEGIN ".reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;" SVDQ_ELECT_END ::"r"(d_tmem),
+               "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+               : "memory");
+}
+
+__device__ __forceinline__ void e_mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(SVDQ_ELECT_BEGIN ".reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;" SVDQ_ELECT_END ::"r"(d_tmem),
+               "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+               : "memory");
+}
+
+__device__ __forceinline__ void e_mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(SVDQ_ELECT_BEGIN ".reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "@e tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;" SVDQ_ELECT_END ::
+                   "r"(d_tmem),
+               "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+               : "memory");
+}
+
+__device__ __forceinline__ void e_commit(uint32_t bar) {
+  asm volatile(SVDQ_ELECT_BEGIN "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" SVDQ_ELECT_END ::
+                   "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void e_commit_pair_both(uint32_t bar) {
+  asm volatile(SVDQ_ELECT_BEGIN
+               "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+               " [%0], %1;" SVDQ_ELECT_END ::"r"(bar),
+               "h"(static_cast<uint16_t>(3))
+               : "memory");
+}
+
+// Warp-uniform bounded waits: every lane polls, lane 0's outcome decides for
+// the whole warp (a warp that issues through elect.sync must stay converged).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns, unsigned int where) {
+  const bool ok = mbar_wait(bar, parity, timeout_ns, where);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+__device__ __forceinline__ bool warp_wait_cluster(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
+                                                  unsigned int where) {
+  const bool ok = mbar_wait_cluster(bar, parity, timeout_ns, where);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+__device__ __forceinline__ bool warp_flag(const volatile int* flag) {
+  return __shfl_sync(0xffffffffu, *flag, 0) != 0;
+}
+
+__device__ __forceinline__ void e_tma_load_3d_pair(uint32_t dst, const void* tmap, uint32_t bar_cluster, int x,
+                                                   int y, int z) {
+  asm volatile(SVDQ_ELECT_BEGIN
+               "@e cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+               " [%0], [%1, {%2, %3, %4}], [%5];" SVDQ_ELECT_END ::"r"(dst),
+               "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(bar_cluster)
+               : "memory");
+}
+
+// Copy 32 rows x 128 bits from shared memory into tensor memory, replicated
+// into the four 32-lane quadrants, in both CTAs of the pair (each from its
+// own shared memory at the same offset).
+__device__ __forceinline__ void e_tmem_cp_pair_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile(SVDQ_ELECT_BEGIN "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" SVDQ_ELECT_END ::"r"(taddr),
+               "l"(sdesc)
+               : "memory");
+}
+
+// TMA store of a 2-D box from shared memory (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(tmap), "r"(src),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until at most N bulk groups of this thread still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void bulk_wait_group() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // ------------------------------------------------------------- clusters --

@@ -217,9 +217,28 @@ int svdq_linear(const uint8_t* x_codes, const uint8_t* x_scales, const void* T, 
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(K / 2), static_cast<uint64_t>(N)};
     const uint64_t strides[1] = {static_cast<uint64_t>(K / 2)};
-    const uint32_t box[2] = {128, 256};
+    const uint32_t box[2] = {128, 128};  // each CTA of a pair loads 128 R rows
     int rc = make_tmap(&tm_rc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, r_codes, dims, strides, box,
                        CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+  }
+  // scale tiles viewed as [tiles][2][256] bytes: a box of 4 tiles is the
+  // 2 KB of scales of one 256-wide K stage of a 128-row band
+  CUtensorMap tm_xs, tm_rs;
+  {
+    const uint64_t dims[3] = {256, 2, static_cast<uint64_t>((M + 127) / 128) * static_cast<uint64_t>(K / 64)};
+    const uint64_t strides[2] = {256, 512};
+    const uint32_t box[3] = {256, 2, 4};
+    int rc = make_tmap(&tm_xs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, x_scales, dims, strides, box,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc) return rc;
+  }
+  {
+    const uint64_t dims[3] = {256, 2, static_cast<uint64_t>((N + 127) / 128) * static_cast<uint64_t>(K / 64)};
+    const uint64_t strides[2] = {256, 512};
+    const uint32_t box[3] = {256, 2, 4};
+    int rc = make_tmap(&tm_rs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, r_scales, dims, strides, box,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
     if (rc) return rc;
   }
   if (r > 0) {
@@ -240,9 +259,17 @@ int svdq_linear(const uint8_t* x_codes, const uint8_t* x_scales, const void* T, 
     std::memset(&tm_l2, 0, sizeof(tm_l2));
   }
 
+  CUtensorMap tm_y;
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(M)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(N) * 2};
+    const uint32_t box[2] = {64, 32};  // one epilogue warp's 32 x 64 block
+    int rc = make_tmap(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, dims, strides, box,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+  }
+
   svdq::LinParams p;
-  p.x_scales = x_scales;
-  p.r_scales = r_scales;
   p.bias = static_cast<const __nv_bfloat16*>(bias);
   p.Y = static_cast<__nv_bfloat16*>(Y);
   p.M = static_cast<int>(M);
@@ -253,15 +280,29 @@ int svdq_linear(const uint8_t* x_codes, const uint8_t* x_scales, const void* T, 
   p.m_tiles = static_cast<int>((M + svdq::kLinBM - 1) / svdq::kLinBM);
   p.tiles = p.m_tiles * static_cast<int>((N + svdq::kLinBN - 1) / svdq::kLinBN);
 
-  const size_t smem = 1024 + svdq::kLinBarOffset + 16 * 8 + 16;
-  if (cudaFuncSetAttribute(svdq::linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
+  const size_t smem = 1024 + svdq::kLinBarOffset + (svdq::kLinNumBars + 2) * 8;
+  const bool full_k = (K % svdq::kLinBK) == 0;
+  auto kern = full_k ? svdq::linear_kernel<true> : svdq::linear_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
     return SVDQ_ERR_CUDA;
   const int sms = sm_count();
-  if (sms <= 0) return SVDQ_ERR_CUDA;
-  dim3 grid(static_cast<unsigned>(p.tiles < sms ? p.tiles : sms));
-  svdq::linear_kernel<<<grid, svdq::kLinThreads, smem, static_cast<cudaStream_t>(stream)>>>(
-      tm_xc, tm_rc, tm_t, tm_l2, p);
+  if (sms < 2) return SVDQ_ERR_CUDA;
+  const int pairs = p.tiles < sms / 2 ? p.tiles : sms / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(svdq::kLinThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tm_xc, tm_rc, tm_xs, tm_rs, tm_t, tm_l2, tm_y, p) != cudaSuccess)
+    return SVDQ_ERR_CUDA;
   return launch_status();
 }
 
