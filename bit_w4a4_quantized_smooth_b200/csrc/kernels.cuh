@@ -106,37 +106,64 @@ __global__ void __launch_bounds__(kPackThreads) pack_residual_kernel(const float
 }
 
 // ============================================ activation quantise + T =====
-// grid (ks, ceil(M/128)) with clusters of ks CTAs along x; 288 threads:
-// warps 0-7 quantise, warp 8 is the producer and MMA issuer.
-// CTA (q, b) handles rows [128 b, 128 b + 128) and K-chunks
-// [q * cpc, (q + 1) * cpc) of 64 columns.  Per chunk, in a 4-stage ring:
-//   warp 8 loads by TMA the X tile (128 rows x 128 B, 128-byte swizzle), the
-//   matching 64 x r rows of L1 (8-column core-matrix interleave) and the 64
-//   inv_lambda values (bulk copy);
-//   quantising thread t handles row t % 128, columns 32 (t / 128) .. + 32 (two
-//   NVFP4 groups): codes and scales go to global memory and bf16(Xh) back into
-//   the swizzled tile in place, which makes it the K-major A operand;
-//   warp 8 then issues four tcgen05 bf16 MMAs (M = 128, N = r, K = 16) adding
-//   Xh L1 into an fp32 [128 x r] tensor-memory accumulator and, once they
-//   have read the stage, refills it.
-// The ks partial T tiles are summed in a fixed order across the cluster
-// through distributed shared memory and rounded once to bf16.
-constexpr int kQaCompute = 256;
-constexpr int kQaThreads = kQaCompute + 32;
-constexpr int kQaStages = 4;
-constexpr uint32_t kQaXBytes = 16384;
+// One CTA per tile of `rows` consecutive rows of X (rows in {16, 32, .., 128},
+// chosen so that the tiles fill the SMs once), over all of K: no split of the
+// reduction, hence no partial sums to combine across CTAs.  704 threads:
+// warps 0-15 quantise (two teams of 8 taking alternate stages), warp 16 is the
+// TMA producer, warp 17 owns the tensor memory and issues the MMAs (both
+// issue warp-wide through elect.sync), warps 18-21 keep the fp32 sum of T.
+// A stage covers 128 columns of K (two 64-column atoms) in a ring of up to 8:
+//   L1 rows [k, k + 128) as two MN-major 128-byte-swizzled atoms of 64 (r) x
+//   64 (k) (a second r-atom when r > 64; columns >= r arrive as zeros);
+//   the X tile, rows x 128 columns as two K-major 128-byte-swizzled atoms;
+//   the 128 inv_lambda values (bulk copy).
+// Warp w of a team quantises group w % 8 (16 columns) of every row, one row
+// per lane: codes and scale go to global memory, bf16(Xh) back into the
+// swizzled tile in place.
+// The MMA warp then adds T^T += L1^T Xh^T with tcgen05 bf16 MMAs (M = 128
+// lanes of TMEM = the columns of L1, N = rows, K = 16): the row tile is the N
+// side, so any multiple of 16 rows is a valid tile.  When r <= 64 the upper
+// 64 lanes of A come from a zeroed shared-memory atom.
+// The tensor cores' accumulation over a long K loses precision (measured: an
+// error growing about linearly with K, biased towards zero, several bf16 ulps
+// of small T entries at K = 12288), so every kQaPromote stages the partial
+// product (K = 256) goes to one of two tensor-memory blocks, and warps 18-21
+// add it into an fp32 running sum on the CUDA cores (fixed order: block 0, 1,
+// ...), overlapping the next block's MMAs.  With the last block they write T
+// rows as bf16 (lane j of the accumulator = column j of T).
+constexpr int kQaQuantWarps = 16;
+constexpr int kQaThreads = kQaQuantWarps * 32 + 64 + 128;
+constexpr int kQaPromote = 2;  // stages (of 128 columns) per tensor-core partial sum
+constexpr int kQaMaxStages = 8;
+constexpr int kQaMaxRows = 128;
+constexpr uint32_t kQaZeroBytes = 8192;
+constexpr uint32_t kQaBarBytes = 256;
+constexpr uint32_t kQaSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory
 
 struct QaParams {
   const float* inv_lambda;
   uint8_t* x_codes;
   uint8_t* x_scales;
   __nv_bfloat16* T;
-  int M, K, r, cpc, ks;
+  int M, K, r, rows, stages, m_pad;
+  uint32_t stage_bytes;
   uint64_t timeout_ns;
 };
 
-__host__ __device__ constexpr uint32_t qa_stage_bytes(int r) {
-  return kQaXBytes + static_cast<uint32_t>(r) * 128u + 1024u;  // X | L1 | inv_lambda (padded)
+// L1 bytes of a stage: two k-atoms of one (r <= 64) or two (r > 64) 8 KB r-atoms
+__host__ __device__ constexpr uint32_t qa_l1_bytes(int r) {
+  return r == 0 ? 0u : (r > 64 ? 32768u : 16384u);
+}
+__host__ __device__ constexpr uint32_t qa_stage_bytes(int r, int rows) {
+  return (qa_l1_bytes(r) + 2u * static_cast<uint32_t>(rows) * 128u + 512u + 1023u) & ~1023u;
+}
+__host__ __device__ constexpr uint32_t qa_zero_bytes(int r) {
+  return (r > 0 && r <= 64) ? kQaZeroBytes : 0u;
+}
+
+// Byte offset of the scale of (row, group g) in the block-scale tile layout.
+__device__ __forceinline__ size_t scale_byte_offset(int row, int g, int K) {
+  return scale_word_offset(row, g & ~3, K) + (g & 3);
 }
 
 __global__ void __launch_bounds__(kQaThreads, 1)
@@ -147,39 +174,56 @@ __global__ void __launch_bounds__(kQaThreads, 1)
                                              ~uintptr_t(1023));
   const int r = p.r;
   const bool has_lr = r > 0;
-  const uint32_t l1_bytes = static_cast<uint32_t>(r) * 128u;
-  const uint32_t stage_bytes = qa_stage_bytes(r);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kQaStages * stage_bytes);
-  uint64_t* full = bars;                    // TMA landed
-  uint64_t* quant = bars + kQaStages;       // 8 quantising warps done with the stage
-  uint64_t* freed = bars + 2 * kQaStages;   // MMAs done reading the stage
-  uint64_t* fin = bars + 3 * kQaStages;     // every MMA of the CTA complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+  const int S = p.stages;
+  const int rows = p.rows;
+  const int K = p.K;
+  const uint32_t stage_bytes = p.stage_bytes;
+  const uint32_t l1_bytes = qa_l1_bytes(r);
+  const uint32_t katom_l1 = l1_bytes / 2;
+  const uint32_t x_atom = static_cast<uint32_t>(rows) * 128u;
+  const uint32_t x_bytes = 2u * x_atom;
+  uint8_t* zero = smem + S * stage_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(zero + qa_zero_bytes(r));
+  uint64_t* full = bars;               // TMA landed
+  uint64_t* quant = bars + S;          // 8 quantising warps done with the stage
+  uint64_t* freed = bars + 2 * S;      // MMAs done reading the stage
+  uint64_t* fin = bars + 3 * S;        // every MMA of the CTA complete
+  uint64_t* acc_full = fin + 1;        // [2] a block's partial product is in tensor memory
+  uint64_t* acc_empty = fin + 3;       // [2] ... and has been added into the running sum
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int row0 = blockIdx.y * 128;
-  const int rank = blockIdx.x;
-  const int nch = p.cpc;
-  const int kc0 = rank * nch;
-  const int K = p.K;
-  const uint32_t tmem_cols = r <= 32 ? 32u : (r <= 64 ? 64u : 128u);
+  const int row0 = blockIdx.x * rows;
+  const int nst = (K / 64 + 1) / 2;  // stages of 128 columns; the last may hold one atom
+  // tensor memory: running sum at column 0, partial-product blocks at RW, 2 RW
+  const uint32_t RW = rows <= 32 ? 32u : (rows <= 64 ? 64u : 128u);
+  const uint32_t tmem_cols = 4 * RW;
+  const int nblk = (nst + kQaPromote - 1) / kQaPromote;
 
-  if (warp == 8 && has_lr) {
+  if (warp == 17 && has_lr) {
     tmem_alloc(smem_u32(tmem_slot), tmem_cols);
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int s = 0; s < kQaStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&quant[s]), kQaCompute / 32);
+      mbar_init(smem_u32(&quant[s]), kQaQuantWarps / 2);
       mbar_init(smem_u32(&freed[s]), 1);
     }
     mbar_init(smem_u32(fin), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&acc_full[b]), 1);
+      mbar_init(smem_u32(&acc_empty[b]), 4);
+    }
     *abort_flag = 0;
     fence_barrier_init();
+  }
+  if (qa_zero_bytes(r) && tid < static_cast<int>(kQaZeroBytes / 16)) {
+    reinterpret_cast<uint4*>(zero)[tid] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -187,174 +231,199 @@ __global__ void __launch_bounds__(kQaThreads, 1)
   const uint32_t tmem = has_lr ? *tmem_slot : 0u;
   const uint32_t smem_base = smem_u32(smem);
 
-  if (warp == 8) {
+  if (warp == 16) {
+    // --------------------------------------------------------- producer --
     if (lane == 0) {
-      // ------------------------------------------- producer + MMA issuer --
       prefetch_tmap(&tm_x);
       if (has_lr) prefetch_tmap(&tm_l1);
-      auto issue = [&](int c) {
-        const int s = c % kQaStages;
-        const int k = (kc0 + c) * 64;
-        const uint32_t fb = smem_u32(&full[s]);
-        const uint32_t dst = smem_base + s * stage_bytes;
-        mbar_arrive_expect_tx(fb, kQaXBytes + l1_bytes + 256u);
-        tma_load_2d(dst, &tm_x, fb, k, row0);
-        if (has_lr) tma_load_3d(dst + kQaXBytes, &tm_l1, fb, 0, k, 0);
-        bulk_load(dst + kQaXBytes + l1_bytes, p.inv_lambda + k, 256u, fb);
-      };
-      int issued = 0;
-      for (int c = 0; c < nch && c < kQaStages; ++c, ++issued) issue(c);
-      // bf16 MMA, M = 128, N = r, A K-major (swizzled X tile), B N-major (L1)
-      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
-                             (static_cast<uint32_t>(r >> 3) << 17) | (8u << 24);
-      for (int c = 0; c < nch; ++c) {
-        const int s = c % kQaStages;
-        const uint32_t ph = (c / kQaStages) & 1;
-        if (*abort_flag) break;
-        if (!mbar_wait(smem_u32(&quant[s]), ph, p.timeout_ns, 10)) {
+    }
+    __syncwarp();
+    int issued = 0;
+    for (int c = 0; c < nst; ++c) {
+      const int s = c % S;
+      if (c >= S) {
+        // the stage's previous chunk: MMAs done reading it (or, without a
+        // low-rank branch, its quantisers done)
+        if (!warp_wait(smem_u32(&freed[s]), ((c / S) - 1) & 1, p.timeout_ns, 11)) {
           *abort_flag = 1;
           break;
         }
+      }
+      const int k = c * 128;
+      const int na = K - k >= 128 ? 2 : 1;  // 64-column atoms in this stage
+      const uint32_t fb = smem_u32(&full[s]);
+      const uint32_t dst = smem_base + s * stage_bytes;
+      e_arrive_expect_tx(fb, na * (katom_l1 + x_atom + 256u));
+      for (int a = 0; a < na; ++a) {
+        e_tma_load_2d(dst + l1_bytes + a * x_atom, &tm_x, fb, k + 64 * a, row0);
         if (has_lr) {
-          tc_fence_after();
-          const uint32_t a0 = smem_base + s * stage_bytes;
-          const uint32_t b0 = a0 + kQaXBytes;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem, make_sdesc(a0 + kk * 32, 16, 1024, 2), make_sdesc(b0 + kk * 256, 128, 1024, 0),
-                     idesc, (c > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(smem_u32(&freed[s]));
-        } else {
-          mbar_arrive(smem_u32(&freed[s]));
-        }
-        if (c + kQaStages < nch) {
-          if (!mbar_wait(smem_u32(&freed[s]), ph, p.timeout_ns, 11)) {
-            *abort_flag = 1;
-            break;
-          }
-          issue(c + kQaStages);
-          ++issued;
+          e_tma_load_2d(dst + a * katom_l1, &tm_l1, fb, 0, k + 64 * a);
+          if (r > 64) e_tma_load_2d(dst + a * katom_l1 + 8192u, &tm_l1, fb, 64, k + 64 * a);
         }
       }
-      if (*abort_flag)  // let this CTA's own copies land before it can exit
-        for (int c = issued > kQaStages ? issued - kQaStages : 0; c < issued; ++c)
-          mbar_wait(smem_u32(&full[c % kQaStages]), (c / kQaStages) & 1, p.timeout_ns, 14);
-      if (has_lr) tc_commit(smem_u32(fin));
+      e_bulk_load(dst + l1_bytes + x_bytes, p.inv_lambda + k, na * 256u, fb);
+      ++issued;
+    }
+    if (warp_flag(abort_flag))  // let this CTA's own copies land before it can exit
+      for (int c = issued > S ? issued - S : 0; c < issued; ++c)
+        warp_wait(smem_u32(&full[c % S]), (c / S) & 1, p.timeout_ns, 14);
+  } else if (warp == 17) {
+    // ------------------------------------------------------- MMA issuer --
+    // bf16 x bf16 -> fp32, A = L1^T MN-major, B = Xh K-major, M = 128, N = rows
+    const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) |
+                           (static_cast<uint32_t>(rows >> 3) << 17) | (8u << 24);
+    const uint32_t zero_addr = smem_u32(zero);
+    for (int c = 0; c < nst; ++c) {
+      const int s = c % S;
+      const int b = c / kQaPromote;
+      const uint32_t buf = b & 1;
+      const bool first = c % kQaPromote == 0;
+      if (warp_flag(abort_flag)) break;
+      if (has_lr && first && b >= 2 &&
+          !warp_wait(smem_u32(&acc_empty[buf]), ((b >> 1) - 1) & 1, p.timeout_ns, 15)) {
+        *abort_flag = 1;
+        break;
+      }
+      if (!warp_wait(smem_u32(&quant[s]), (c / S) & 1, p.timeout_ns, 10)) {
+        *abort_flag = 1;
+        break;
+      }
+      if (has_lr) {
+        tc_fence_after();
+        const uint32_t d = tmem + RW * (1 + buf);
+        const int na = K - c * 128 >= 128 ? 2 : 1;
+        const uint32_t st = smem_base + s * stage_bytes;
+        for (int a = 0; a < na; ++a) {
+          const uint32_t l1a = st + a * katom_l1;
+          const uint32_t xa = st + l1_bytes + a * x_atom;
+          // second r-atom (A rows 64..127): loaded for r > 64, else the zero atom
+          const uint32_t lbo = r > 64 ? 8192u : zero_addr - l1a;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            e_mma_bf16(d, make_sdesc(l1a + kk * 2048, lbo, 1024, 2), make_sdesc(xa + kk * 32, 16, 1024, 2),
+                       idesc, (first && (a | kk) == 0) ? 0u : 1u);
+        }
+        e_commit(smem_u32(&freed[s]));
+        if (c % kQaPromote == kQaPromote - 1 || c == nst - 1) e_commit(smem_u32(&acc_full[buf]));
+      } else {
+        e_arrive(smem_u32(&freed[s]));
+      }
+    }
+    if (has_lr) e_commit(smem_u32(fin));
+  } else if (warp >= 18) {
+    // ------------------------------------------- fp32 running sum of T --
+    const int q = warp & 3;  // tensor-memory lane quadrant of this warp
+    const bool active = 32 * q < r;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+    const int j = 32 * q + lane;  // column of T held by this lane
+    for (int b = 0; has_lr && b < nblk; ++b) {
+      const uint32_t buf = b & 1;
+      if (!warp_wait(smem_u32(&acc_full[buf]), (b >> 1) & 1, p.timeout_ns, 16)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      if (active) {
+        const bool last = b == nblk - 1;
+        for (int n0 = 0; n0 < rows; n0 += 16) {
+          uint32_t v[16], t[16];
+          tmem_ld_32x32b_x16(tmem + lane_base + RW * (1 + buf) + n0, v);
+          if (b > 0) tmem_ld_32x32b_x16(tmem + lane_base + n0, t);
+          tmem_ld_wait();
+          if (b > 0) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              v[i] = __float_as_uint(__fadd_rn(__uint_as_float(t[i]), __uint_as_float(v[i])));
+          }
+          if (!last) {
+            tmem_st_32x32b_x16(tmem + lane_base + n0, v);
+          } else if (j < r) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int m = row0 + n0 + i;
+              if (m < p.M) p.T[static_cast<size_t>(m) * r + j] = __float2bfloat16_rn(__uint_as_float(v[i]));
+            }
+          }
+        }
+        if (!last) tmem_st_wait();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[buf]));
     }
   } else {
     // ------------------------------------------------------- quantisers --
-    const int rr = tid & 127;  // row inside the tile
-    const int h = tid >> 7;    // which 32-column half of the chunk
-    const int m = row0 + rr;
-    const int sw = rr & 7;     // 128-byte swizzle phase of the row
-    for (int c = 0; c < nch; ++c) {
-      const int s = c % kQaStages;
-      const uint32_t ph = (c / kQaStages) & 1;
+    const int team = warp >> 3;
+    const int g = warp & 7;  // the 16-column group of each stage this warp quantises
+    for (int c = team; c < nst; c += 2) {
+      const int s = c % S;
       // warp-uniform outcome: the warp meets __syncwarp below together
-      const bool ok = !warp_flag(abort_flag) && warp_wait(smem_u32(&full[s]), ph, p.timeout_ns, 12);
+      const bool ok = !warp_flag(abort_flag) && warp_wait(smem_u32(&full[s]), (c / S) & 1, p.timeout_ns, 12);
       if (!ok) {
         *abort_flag = 1;
         break;
       }
-      const int k = (kc0 + c) * 64;
-      uint8_t* stage = smem + s * stage_bytes;
-      uint8_t* row = stage + rr * 128;
-      const float4* il = reinterpret_cast<const float4*>(stage + kQaXBytes + l1_bytes) + 8 * h;
-      uint32_t cw[4];
-      uint32_t swd = 0;
-#pragma unroll
-      for (int g = 0; g < 2; ++g) {
-        const int j0 = 4 * h + 2 * g;  // logical 16-byte chunk of the row
-        uint4 w0 = *reinterpret_cast<const uint4*>(row + ((j0 ^ sw) << 4));
-        uint4 w1 = *reinterpret_cast<const uint4*>(row + (((j0 + 1) ^ sw) << 4));
-        const float4 l0 = il[4 * g + 0], l1 = il[4 * g + 1], l2 = il[4 * g + 2], l3 = il[4 * g + 3];
-        float v[16];
-        v[0] = __fmul_rn(bf16_lo(w0.x), l0.x);  v[1] = __fmul_rn(bf16_hi(w0.x), l0.y);
-        v[2] = __fmul_rn(bf16_lo(w0.y), l0.z);  v[3] = __fmul_rn(bf16_hi(w0.y), l0.w);
-        v[4] = __fmul_rn(bf16_lo(w0.z), l1.x);  v[5] = __fmul_rn(bf16_hi(w0.z), l1.y);
-        v[6] = __fmul_rn(bf16_lo(w0.w), l1.z);  v[7] = __fmul_rn(bf16_hi(w0.w), l1.w);
-        v[8] = __fmul_rn(bf16_lo(w1.x), l2.x);  v[9] = __fmul_rn(bf16_hi(w1.x), l2.y);
-        v[10] = __fmul_rn(bf16_lo(w1.y), l2.z); v[11] = __fmul_rn(bf16_hi(w1.y), l2.w);
-        v[12] = __fmul_rn(bf16_lo(w1.z), l3.x); v[13] = __fmul_rn(bf16_hi(w1.z), l3.y);
-        v[14] = __fmul_rn(bf16_lo(w1.w), l3.z); v[15] = __fmul_rn(bf16_hi(w1.w), l3.w);
-        swd |= nvfp4_group(v, cw[2 * g], cw[2 * g + 1]) << (8 * g);
-        if (has_lr) {
-          w0 = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                          pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-          w1 = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
-                          pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
-          *reinterpret_cast<uint4*>(row + ((j0 ^ sw) << 4)) = w0;
-          *reinterpret_cast<uint4*>(row + (((j0 + 1) ^ sw) << 4)) = w1;
+      const int k = c * 128;
+      const int ng = K - k >= 128 ? 8 : 4;  // groups per row in this stage
+      if (g < ng) {
+        uint8_t* stage = smem + s * stage_bytes;
+        const float4* lam = reinterpret_cast<const float4*>(stage + l1_bytes + x_bytes) + 4 * g;
+        const float4 l0 = lam[0], l1 = lam[1], l2 = lam[2], l3 = lam[3];
+        const int kg = k + 16 * g;
+        const int j0 = (g & 3) * 2;  // logical 16-byte chunk of the row
+        uint8_t* atom = stage + l1_bytes + (g >> 2) * x_atom;
+        for (int rr = lane; rr < rows; rr += 32) {
+          uint8_t* row = atom + rr * 128;
+          const int sw = rr & 7;  // 128-byte swizzle phase of the row
+          uint4 w0 = *reinterpret_cast<const uint4*>(row + ((j0 ^ sw) << 4));
+          uint4 w1 = *reinterpret_cast<const uint4*>(row + (((j0 + 1) ^ sw) << 4));
+          float v[16];
+          v[0] = __fmul_rn(bf16_lo(w0.x), l0.x);  v[1] = __fmul_rn(bf16_hi(w0.x), l0.y);
+          v[2] = __fmul_rn(bf16_lo(w0.y), l0.z);  v[3] = __fmul_rn(bf16_hi(w0.y), l0.w);
+          v[4] = __fmul_rn(bf16_lo(w0.z), l1.x);  v[5] = __fmul_rn(bf16_hi(w0.z), l1.y);
+          v[6] = __fmul_rn(bf16_lo(w0.w), l1.z);  v[7] = __fmul_rn(bf16_hi(w0.w), l1.w);
+          v[8] = __fmul_rn(bf16_lo(w1.x), l2.x);  v[9] = __fmul_rn(bf16_hi(w1.x), l2.y);
+          v[10] = __fmul_rn(bf16_lo(w1.y), l2.z); v[11] = __fmul_rn(bf16_hi(w1.y), l2.w);
+          v[12] = __fmul_rn(bf16_lo(w1.z), l3.x); v[13] = __fmul_rn(bf16_hi(w1.z), l3.y);
+          v[14] = __fmul_rn(bf16_lo(w1.w), l3.z); v[15] = __fmul_rn(bf16_hi(w1.w), l3.w);
+          uint32_t lo, hi;
+          const uint32_t sc = nvfp4_group(v, lo, hi);
+          if (has_lr) {
+            w0 = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+            w1 = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                            pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+            *reinterpret_cast<uint4*>(row + ((j0 ^ sw) << 4)) = w0;
+            *reinterpret_cast<uint4*>(row + (((j0 + 1) ^ sw) << 4)) = w1;
+          }
+          const int m = row0 + rr;
+          if (m < p.M)
+            *reinterpret_cast<uint2*>(p.x_codes + static_cast<size_t>(m) * (K >> 1) + (kg >> 1)) =
+                make_uint2(lo, hi);
+          if (m < p.m_pad) p.x_scales[scale_byte_offset(m, kg >> 4, K)] = static_cast<uint8_t>(sc);
         }
       }
-      if (m < p.M)
-        *reinterpret_cast<uint4*>(p.x_codes + static_cast<size_t>(m) * (K >> 1) + (k >> 1) + 16 * h) =
-            make_uint4(cw[0], cw[1], cw[2], cw[3]);
-      *reinterpret_cast<uint16_t*>(p.x_scales + scale_word_offset(m, k >> 4, K) + 2 * h) =
-          static_cast<uint16_t>(swd);
       if (has_lr) fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&quant[s]));
+    }
+    // scale-layout padding rows that no tile covers: zero scales
+    const int covered = gridDim.x * rows;
+    if (blockIdx.x == gridDim.x - 1 && covered < p.m_pad) {
+      const int gk = K >> 4;
+      for (int i = tid; i < (p.m_pad - covered) * gk; i += kQaQuantWarps * 32)
+        p.x_scales[scale_byte_offset(covered + i / gk, i % gk, K)] = 0;
     }
   }
 
   if (has_lr) {
     // every MMA of this CTA (also after an abort) completes before the
-    // accumulator is read or the tensor memory released
-    const bool ok = mbar_wait(smem_u32(fin), 0, p.timeout_ns, 13);
-    if (!ok) *abort_flag = 1;
-    __syncthreads();
-    tc_fence_after();
-    const bool good = !*abort_flag;
-    float* part = reinterpret_cast<float*>(smem);  // ring is idle: reuse it
-    if (warp < 4 && good) {
-      const int m = row0 + tid;
-      const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-      for (int c0 = 0; c0 < r; c0 += 16) {
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(tmem + lane_base + c0, v);
-        tmem_ld_wait();
-        if (p.ks == 1) {
-          if (m < p.M) {
-            uint4* dst = reinterpret_cast<uint4*>(p.T + static_cast<size_t>(m) * r + c0);
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-              dst[j] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
-                                  pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
-                                  pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
-                                  pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; j += 4)
-            *reinterpret_cast<uint4*>(part + tid * r + c0 + j) = make_uint4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-        }
-      }
-    }
-    if (p.ks > 1) {
-      cluster_sync();
-      const int rows_per = 128 / p.ks;
-      const int q4 = r >> 2;
-      const uint32_t part_s = smem_u32(part);
-      for (int it = tid; it < rows_per * q4; it += kQaThreads) {
-        const int rr = rank * rows_per + it / q4;
-        const int j = (it % q4) * 4;
-        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int src = 0; src < p.ks; ++src) {
-          const float4 v = ld_shared_cluster_f4(map_shared_rank(part_s + (rr * r + j) * 4, src));
-          sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
-        }
-        const int mm = row0 + rr;
-        if (good && mm < p.M)
-          *reinterpret_cast<uint2*>(p.T + static_cast<size_t>(mm) * r + j) =
-              make_uint2(pack_bf16x2(sum.x, sum.y), pack_bf16x2(sum.z, sum.w));
-      }
-      cluster_sync();
-    }
+    // tensor memory is released
+    if (!mbar_wait(smem_u32(fin), 0, p.timeout_ns, 13)) *abort_flag = 1;
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 8 && has_lr) tmem_dealloc(tmem, tmem_cols);
+  if (warp == 17 && has_lr) tmem_dealloc(tmem, tmem_cols);
 }
 
 // ================================================== fused 4-bit linear ====

@@ -15,7 +15,6 @@
 
 namespace {
 
-using svdq::kQaStages;
 
 uint64_t g_timeout_ns = 0;
 std::once_flag g_timeout_once;
@@ -80,15 +79,14 @@ int sm_count() {
   return cached[dev];
 }
 
-// Largest cluster size (1, 2, 4, 8) dividing the number of 64-column chunks
-// such that row tiles x cluster stays within about two waves of 148 SMs.
-int choose_ks(int64_t M, int64_t K) {
-  const int64_t tiles = (M + 127) / 128;
-  const int64_t chunks = K / 64;
-  int ks = 1;
-  for (int c : {2, 4, 8})
-    if (chunks % c == 0 && tiles * c <= 2 * 148) ks = c;
-  return ks;
+// Rows per activation tile: a multiple of 16 in [16, 128] such that the
+// tiles cover M in about one wave over the SMs (one CTA per SM).
+int choose_rows(int64_t M, int sms) {
+  int64_t rows = (M + sms - 1) / sms;
+  rows = (rows + 15) / 16 * 16;
+  if (rows < 16) rows = 16;
+  if (rows > svdq::kQaMaxRows) rows = svdq::kQaMaxRows;
+  return static_cast<int>(rows);
 }
 
 }  // namespace
@@ -135,29 +133,36 @@ int svdq_quantize_act(const void* X, const float* inv_lambda, const void* L1, in
       (r > 0 && (!aligned16(L1) || !aligned16(T))))
     return SVDQ_ERR_MISALIGNED;
 
+  const int sms = sm_count();
+  if (sms <= 0) return SVDQ_ERR_CUDA;
+  const int rows = choose_rows(M, sms);
   CUtensorMap tm_x, tm_l1;
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
     const uint64_t strides[1] = {static_cast<uint64_t>(K) * 2};
-    const uint32_t box[2] = {64, 128};
+    const uint32_t box[2] = {64, static_cast<uint32_t>(rows)};
     int rc = make_tmap(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, dims, strides, box,
                        CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
   }
   if (r > 0) {
-    // L1 [K][r] viewed as [r/8][K][8]: boxes of 8 columns x 64 rows give the
-    // 8 x 16-byte core matrices of an N-major operand without swizzle.
-    const uint64_t dims[3] = {8, static_cast<uint64_t>(K), static_cast<uint64_t>(r / 8)};
-    const uint64_t strides[2] = {static_cast<uint64_t>(r) * 2, 16};
-    const uint32_t box[3] = {8, 64, static_cast<uint32_t>(r / 8)};
-    int rc = make_tmap(&tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, L1, dims, strides, box,
-                       CU_TENSOR_MAP_SWIZZLE_NONE);
+    // L1 [K][r]: boxes of 64 (r, zero-filled past r) x 64 (k) with 128-byte
+    // swizzle are the MN-major atoms of the A operand L1^T.
+    const uint64_t dims[2] = {static_cast<uint64_t>(r), static_cast<uint64_t>(K)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(r) * 2};
+    const uint32_t box[2] = {64, 64};
+    int rc = make_tmap(&tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L1, dims, strides, box,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
   } else {
     std::memset(&tm_l1, 0, sizeof(tm_l1));
   }
 
-  const int ks = choose_ks(M, K);
+  const uint32_t stage_bytes = svdq::qa_stage_bytes(static_cast<int>(r), rows);
+  const uint32_t fixed = 1024 + svdq::qa_zero_bytes(static_cast<int>(r)) + svdq::kQaBarBytes;
+  int stages = static_cast<int>((svdq::kQaSmemLimit - fixed) / stage_bytes);
+  if (stages > svdq::kQaMaxStages) stages = svdq::kQaMaxStages;
+  if (stages < 2) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   svdq::QaParams p;
   p.inv_lambda = inv_lambda;
   p.x_codes = x_codes;
@@ -166,27 +171,23 @@ int svdq_quantize_act(const void* X, const float* inv_lambda, const void* L1, in
   p.M = static_cast<int>(M);
   p.K = static_cast<int>(K);
   p.r = static_cast<int>(r);
-  p.ks = ks;
-  p.cpc = static_cast<int>(K / 64 / ks);
+  p.rows = rows;
+  p.stages = stages;
+  p.m_pad = static_cast<int>((M + 127) / 128 * 128);
+  p.stage_bytes = stage_bytes;
   p.timeout_ns = wait_timeout_ns();
 
-  const size_t smem = 1024 + kQaStages * static_cast<size_t>(svdq::qa_stage_bytes(static_cast<int>(r))) +
-                      (3 * kQaStages + 1) * 8 + 16;
+  const size_t smem = fixed + static_cast<size_t>(stages) * stage_bytes;
   if (cudaFuncSetAttribute(svdq::quantize_act_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return SVDQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(ks), static_cast<unsigned>((M + 127) / 128));
+  cfg.gridDim = dim3(static_cast<unsigned>((M + rows - 1) / rows));
   cfg.blockDim = dim3(svdq::kQaThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(ks);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
   if (cudaLaunchKernelEx(&cfg, svdq::quantize_act_kernel, tm_x, tm_l1, p) != cudaSuccess)
     return SVDQ_ERR_CUDA;
   return launch_status();

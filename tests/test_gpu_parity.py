@@ -29,6 +29,7 @@ SMALL = [
     ("flux_qkv", 1, 1024, 256, 64),              # one token
     ("sweep_3072", 128, 2048, 256, 48),          # cluster of 8 along K, r = 48
     ("flux_qkv", 300, 192, 528, 16),             # K = 3 chunks, N tail of 16 columns
+    ("flux_qkv", 160, 384, 256, 96),             # r = 96: second r-atom of L1 partly past r
 ]
 
 
@@ -168,6 +169,7 @@ MULTI = [
     ("flux_qkv", 2048, 256, 5120, 32),
     ("flux_mlp_up", 1536, 512, 8192, 0),
     ("flux_mlp_down", 2500, 320, 4112, 64),   # ragged M, N and K
+    ("sweep_3072", 20000, 256, 256, 32),      # 128-row activation tiles, more tiles than SMs
 ]
 
 
