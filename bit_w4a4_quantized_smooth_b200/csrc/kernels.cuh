@@ -23,6 +23,14 @@
 
 namespace svdq {
 
+// First 1024-byte aligned byte of the dynamic shared memory (128-byte
+// swizzled TMA / MMA tiles need it).  The offset is added to the shared array
+// itself, so the compiler keeps every derived pointer in the shared window
+// (LDS/STS) instead of falling back to generic addressing.
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* smem_raw) {
+  return smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+}
+
 // ------------------------------------------------------ NVFP4 quantiser --
 // One group of 16 fp32 values (NVFP4: E2M1 elements, one unsigned E4M3
 // scale per 16, scale = amax / 6):
@@ -108,36 +116,40 @@ __global__ void __launch_bounds__(kPackThreads) pack_residual_kernel(const float
 // ============================================ activation quantise + T =====
 // One CTA per tile of `rows` consecutive rows of X (rows in {16, 32, .., 128},
 // chosen so that the tiles fill the SMs once), over all of K: no split of the
-// reduction, hence no partial sums to combine across CTAs.  704 threads:
-// warps 0-15 quantise (two teams of 8 taking alternate stages), warp 16 is the
-// TMA producer, warp 17 owns the tensor memory and issues the MMAs (both
-// issue warp-wide through elect.sync), warps 18-21 keep the fp32 sum of T.
-// A stage covers 128 columns of K (two 64-column atoms) in a ring of up to 8:
-//   L1 rows [k, k + 128) as two MN-major 128-byte-swizzled atoms of 64 (r) x
-//   64 (k) (a second r-atom when r > 64; columns >= r arrive as zeros);
-//   the X tile, rows x 128 columns as two K-major 128-byte-swizzled atoms;
-//   the 128 inv_lambda values (bulk copy).
-// Warp w of a team quantises group w % 8 (16 columns) of every row, one row
-// per lane: codes and scale go to global memory, bf16(Xh) back into the
-// swizzled tile in place.
-// The MMA warp then adds T^T += L1^T Xh^T with tcgen05 bf16 MMAs (M = 128
-// lanes of TMEM = the columns of L1, N = rows, K = 16): the row tile is the N
-// side, so any multiple of 16 rows is a valid tile.  When r <= 64 the upper
-// 64 lanes of A come from a zeroed shared-memory atom.
-// The tensor cores' accumulation over a long K loses precision (measured: an
-// error growing about linearly with K, biased towards zero, several bf16 ulps
-// of small T entries at K = 12288), so every kQaPromote stages the partial
-// product (K = 256) goes to one of two tensor-memory blocks, and warps 18-21
-// add it into an fp32 running sum on the CUDA cores (fixed order: block 0, 1,
-// ...), overlapping the next block's MMAs.  With the last block they write T
-// rows as bf16 (lane j of the accumulator = column j of T).
-constexpr int kQaQuantWarps = 16;
-constexpr int kQaThreads = kQaQuantWarps * 32 + 64 + 128;
-constexpr int kQaPromote = 2;  // stages (of 128 columns) per tensor-core partial sum
+// reduction, hence no partial sums to combine across CTAs.  512 threads, all
+// computing; warp 0 also issues the TMA loads (warp-wide, elect.sync), one
+// stage behind the consumers, so that four warps per sub-core keep up to 128
+// registers each.
+//
+// A ring stage holds xw = 512, 256 or 128 columns of the tile (the widest
+// that still leaves a few stages of shared memory): the X atoms (64 columns, K-major, 128-byte swizzle), the matching xw
+// rows of L1 as atoms of aw = r (16 or 32) or 64 columns (32/64/128-byte
+// swizzle, columns past r arrive as zeros) and the inv_lambda values.
+// Per stage every compute warp
+//   1. quantises 16-column groups of 32 rows (one row per lane), two at a time
+//      so that each thread has two independent dependency chains in flight:
+//      codes and scale to global memory, bf16(Xh) back into the X atom in
+//      place;
+//   2. after all 16 warps have written bf16(Xh) (an mbarrier), adds its share
+//      of Xh L1 with warp-level tensor-core MMAs (m16n8k16, bf16 in, fp32 out;
+//      fragments by ldmatrix from the swizzled atoms) into a stage partial,
+//      then folds that partial into fp32 running sums on the CUDA cores.
+// The low-rank contraction (2 rows K r flops) is small and its N = r is at
+// most 128: a tcgen05 kind::f16 MMA costs about 85 cycles whatever its N up
+// to 128 (measured), and one issuing thread per CTA would need K / 16 of them
+// in series, 8 us at K = 3072.  Spread over 16 warps and the four sub-core
+// tensor units it hides under the HBM stream.  Folding each stage's partial
+// (K <= 256) into fp32 keeps long K as accurate as an fp32 sum (tensor-core
+// accumulation over thousands of terms drifts by several bf16 ulps).
+// T tiles (16 x 16) are split over the warps; when there are fewer than 16,
+// several warps share a tile over disjoint k-steps and the partials are summed
+// in a fixed order at the end.
+constexpr int kQaWarps = 16;
+constexpr int kQaThreads = kQaWarps * 32;
 constexpr int kQaMaxStages = 8;
 constexpr int kQaMaxRows = 128;
-constexpr uint32_t kQaZeroBytes = 8192;
-constexpr uint32_t kQaBarBytes = 256;
+constexpr int kQaMaxUnits = 2;  // 16 x 16 T tiles per warp: rows x r <= 8192
+constexpr uint32_t kQaBarBytes = 256 + 512;  // barriers, abort flag, reciprocal table
 constexpr uint32_t kQaSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory
 
 struct QaParams {
@@ -145,20 +157,23 @@ struct QaParams {
   uint8_t* x_codes;
   uint8_t* x_scales;
   __nv_bfloat16* T;
-  int M, K, r, rows, stages, m_pad;
+  int M, K, r, rows, m_pad;
+  int xw;      // columns per stage (512, 256 or 128)
+  int aw;      // columns per L1 atom (16, 32 or 64)
+  int stages;
   uint32_t stage_bytes;
   uint64_t timeout_ns;
 };
 
-// L1 bytes of a stage: two k-atoms of one (r <= 64) or two (r > 64) 8 KB r-atoms
-__host__ __device__ constexpr uint32_t qa_l1_bytes(int r) {
-  return r == 0 ? 0u : (r > 64 ? 32768u : 16384u);
+__host__ __device__ constexpr int qa_xw(int rows, int r) {
+  return (rows <= 32 && r <= 32) ? 512 : ((rows <= 64 && r <= 64) ? 256 : 128);
 }
-__host__ __device__ constexpr uint32_t qa_stage_bytes(int r, int rows) {
-  return (qa_l1_bytes(r) + 2u * static_cast<uint32_t>(rows) * 128u + 512u + 1023u) & ~1023u;
-}
-__host__ __device__ constexpr uint32_t qa_zero_bytes(int r) {
-  return (r > 0 && r <= 64) ? kQaZeroBytes : 0u;
+__host__ __device__ constexpr int qa_aw(int r) { return r <= 16 ? 16 : (r <= 32 ? 32 : 64); }
+__host__ __device__ constexpr int qa_natoms(int r) { return r == 0 ? 0 : (r + qa_aw(r) - 1) / qa_aw(r); }
+__host__ __device__ constexpr uint32_t qa_stage_bytes(int rows, int r) {
+  return (static_cast<uint32_t>(qa_xw(rows, r)) *
+              (2u * static_cast<uint32_t>(rows) + 2u * static_cast<uint32_t>(qa_natoms(r) * qa_aw(r)) + 4u) +
+          1023u) & ~1023u;
 }
 
 // Byte offset of the scale of (row, group g) in the block-scale tile layout.
@@ -166,264 +181,319 @@ __device__ __forceinline__ size_t scale_byte_offset(int row, int g, int K) {
   return scale_word_offset(row, g & ~3, K) + (g & 3);
 }
 
+// (d0, d1) = (a0 * b0, a1 * b1), each rounded to nearest fp32 (packed fp32 pipe).
+__device__ __forceinline__ void mul2_rn(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 __global__ void __launch_bounds__(kQaThreads, 1)
     quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_l1, const QaParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = align_smem_1024(smem_raw);
   const int r = p.r;
   const bool has_lr = r > 0;
-  const int S = p.stages;
   const int rows = p.rows;
   const int K = p.K;
-  const uint32_t stage_bytes = p.stage_bytes;
-  const uint32_t l1_bytes = qa_l1_bytes(r);
-  const uint32_t katom_l1 = l1_bytes / 2;
+  const int xw = p.xw;
+  const int aw = p.aw;
+  const int S = p.stages;
+  const int xa = xw / 64;   // X atoms per stage
+  const int gs = xw / 16;   // 16-column groups per row per stage
   const uint32_t x_atom = static_cast<uint32_t>(rows) * 128u;
-  const uint32_t x_bytes = 2u * x_atom;
-  uint8_t* zero = smem + S * stage_bytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(zero + qa_zero_bytes(r));
-  uint64_t* full = bars;               // TMA landed
-  uint64_t* quant = bars + S;          // 8 quantising warps done with the stage
-  uint64_t* freed = bars + 2 * S;      // MMAs done reading the stage
-  uint64_t* fin = bars + 3 * S;        // every MMA of the CTA complete
-  uint64_t* acc_full = fin + 1;        // [2] a block's partial product is in tensor memory
-  uint64_t* acc_empty = fin + 3;       // [2] ... and has been added into the running sum
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 5);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t x_bytes = xa * x_atom;
+  const uint32_t l1_atom = static_cast<uint32_t>(xw * aw * 2);
+  const int natoms = has_lr ? (r + aw - 1) / aw : 0;
+  const uint32_t l1_bytes = natoms * l1_atom;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * p.stage_bytes);  // [S] stage landed
+  uint64_t* xready = full + S;   // [S] all 16 warps wrote bf16(Xh) of the stage
+  uint64_t* empty = xready + S;  // [S] all 16 warps done with the stage
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + S);
+  float* rcp_tab = reinterpret_cast<float*>(empty + S + 1);  // [128]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int row0 = blockIdx.x * rows;
-  const int nst = (K / 64 + 1) / 2;  // stages of 128 columns; the last may hold one atom
-  // tensor memory: running sum at column 0, partial-product blocks at RW, 2 RW
-  const uint32_t RW = rows <= 32 ? 32u : (rows <= 64 ? 64u : 128u);
-  const uint32_t tmem_cols = 4 * RW;
-  const int nblk = (nst + kQaPromote - 1) / kQaPromote;
+  const int nst = (K + xw - 1) / xw;
 
-  if (warp == 17 && has_lr) {
-    tmem_alloc(smem_u32(tmem_slot), tmem_cols);
-    tmem_relinquish();
-  }
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&quant[s]), kQaQuantWarps / 2);
-      mbar_init(smem_u32(&freed[s]), 1);
-    }
-    mbar_init(smem_u32(fin), 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&acc_full[b]), 1);
-      mbar_init(smem_u32(&acc_empty[b]), 4);
+      mbar_init(smem_u32(&xready[s]), kQaWarps);
+      mbar_init(smem_u32(&empty[s]), kQaWarps);
     }
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (qa_zero_bytes(r) && tid < static_cast<int>(kQaZeroBytes / 16)) {
-    reinterpret_cast<uint4*>(zero)[tid] = make_uint4(0u, 0u, 0u, 0u);
-    fence_proxy_async_smem();
-  }
-  tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = has_lr ? *tmem_slot : 0u;
-  const uint32_t smem_base = smem_u32(smem);
 
-  if (warp == 16) {
-    // --------------------------------------------------------- producer --
+  // T tiles of 16 rows x 16 columns ("units"); see the header comment
+  const int nbr = r / 16;               // 16-column blocks of T
+  const int U = (rows / 16) * nbr;
+  int wpu = 1, kp = 0, nu = 0;
+  if (U >= kQaWarps) {
+    nu = (U - warp + kQaWarps - 1) / kQaWarps;  // units warp, warp + 16, ...
+  } else if (U > 0) {
+    wpu = kQaWarps / U;                  // warps sharing a unit
+    if (warp < U * wpu) {
+      nu = 1;
+      kp = warp / U;
+    }
+  }
+  float tot[kQaMaxUnits][8];
+#pragma unroll
+  for (int i = 0; i < kQaMaxUnits; ++i)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) tot[i][e] = 0.0f;
+
+  // TMA loads of stage c into its ring slot (warp 0, warp-wide)
+  auto load_stage = [&](int c, int slot) {
+    const int k = c * xw;
+    const int na = min(xa, (K - k) / 64);  // X atoms inside K
+    const uint32_t fb = smem_u32(&full[slot]);
+    const uint32_t dst = smem_u32(smem + slot * p.stage_bytes);
+    // L1 boxes hold at most 256 rows (a TMA limit); an atom is xw rows, and
+    // boxes that would start past K are not loaded (no MMA reads them)
+    const int lb = xw < 256 ? xw : 256;
+    const int nlb = (min(xw, K - k) + lb - 1) / lb;
+    e_arrive_expect_tx(fb, na * (x_atom + 256u) + natoms * nlb * lb * aw * 2);
+    for (int a = 0; a < na; ++a) e_tma_load_2d(dst + a * x_atom, &tm_x, fb, k + 64 * a, row0);
+    for (int t = 0; t < natoms; ++t)
+      for (int h = 0; h < nlb; ++h)
+        e_tma_load_2d(dst + x_bytes + t * l1_atom + h * lb * aw * 2, &tm_l1, fb, t * aw, k + h * lb);
+    e_bulk_load(dst + x_bytes + l1_bytes, p.inv_lambda + k, na * 256u, fb);
+  };
+  int issued = 0;
+  if (warp == 0) {
     if (lane == 0) {
       prefetch_tmap(&tm_x);
       if (has_lr) prefetch_tmap(&tm_l1);
     }
     __syncwarp();
-    int issued = 0;
+    for (; issued < S && issued < nst; ++issued) load_stage(issued, issued);
+  }
+  {
+    const int gs_log2 = 31 - __clz(gs);
+    const int items = gs * ((rows + 31) >> 5);  // (group, 32-row block) pairs per stage
+    const int mi = lane >> 3;            // ldmatrix: matrix this lane addresses
+    // reciprocals of the 127 finite E4M3 scale values (0 for the zero scale)
+    if (warp < 4) {
+      const float sd = e4m3_to_f32(static_cast<uint32_t>(tid));
+      rcp_tab[tid] = sd == 0.0f ? 0.0f : __frcp_rn(sd);
+    }
+    __syncthreads();
+    // per-unit constants of the low-rank MMAs (unit u of this warp: slot i)
+    uint32_t a_off[kQaMaxUnits], b_off[kQaMaxUnits];
+    int a_sw[kQaMaxUnits];
+#pragma unroll
+    for (int i = 0; i < kQaMaxUnits; ++i) {
+      const int u = i < nu ? (U >= kQaWarps ? warp + kQaWarps * i : warp % U) : 0;
+      const int rb = nbr ? u / nbr : 0, nb = nbr ? u % nbr : 0;
+      const int arow = rb * 16 + (lane & 7) + ((mi & 1) << 3);
+      a_off[i] = static_cast<uint32_t>(arow * 128);
+      a_sw[i] = arow & 7;
+      const int bn = nb * 16 + ((mi >> 1) << 3);
+      const int bk = (lane & 7) + ((mi & 1) << 3);  // k offset inside a 16-step (swizzle is periodic in 16)
+      const int bsw = aw == 64 ? (bk & 7) : (aw == 32 ? ((bk >> 1) & 3) : ((bk >> 2) & 1));
+      b_off[i] = static_cast<uint32_t>((bn / aw) * l1_atom + bk * (aw * 2) + ((((bn % aw) >> 3) ^ bsw) << 4));
+    }
+    const uint32_t b_kstep = static_cast<uint32_t>(16 * aw * 2);  // bytes of 16 L1 rows
+    int s = 0;
+    uint32_t ph = 0;
     for (int c = 0; c < nst; ++c) {
-      const int s = c % S;
-      if (c >= S) {
-        // the stage's previous chunk: MMAs done reading it (or, without a
-        // low-rank branch, its quantisers done)
-        if (!warp_wait(smem_u32(&freed[s]), ((c / S) - 1) & 1, p.timeout_ns, 11)) {
-          *abort_flag = 1;
-          break;
-        }
-      }
-      const int k = c * 128;
-      const int na = K - k >= 128 ? 2 : 1;  // 64-column atoms in this stage
-      const uint32_t fb = smem_u32(&full[s]);
-      const uint32_t dst = smem_base + s * stage_bytes;
-      e_arrive_expect_tx(fb, na * (katom_l1 + x_atom + 256u));
-      for (int a = 0; a < na; ++a) {
-        e_tma_load_2d(dst + l1_bytes + a * x_atom, &tm_x, fb, k + 64 * a, row0);
-        if (has_lr) {
-          e_tma_load_2d(dst + a * katom_l1, &tm_l1, fb, 0, k + 64 * a);
-          if (r > 64) e_tma_load_2d(dst + a * katom_l1 + 8192u, &tm_l1, fb, 64, k + 64 * a);
-        }
-      }
-      e_bulk_load(dst + l1_bytes + x_bytes, p.inv_lambda + k, na * 256u, fb);
-      ++issued;
-    }
-    if (warp_flag(abort_flag))  // let this CTA's own copies land before it can exit
-      for (int c = issued > S ? issued - S : 0; c < issued; ++c)
-        warp_wait(smem_u32(&full[c % S]), (c / S) & 1, p.timeout_ns, 14);
-  } else if (warp == 17) {
-    // ------------------------------------------------------- MMA issuer --
-    // bf16 x bf16 -> fp32, A = L1^T MN-major, B = Xh K-major, M = 128, N = rows
-    const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) |
-                           (static_cast<uint32_t>(rows >> 3) << 17) | (8u << 24);
-    const uint32_t zero_addr = smem_u32(zero);
-    for (int c = 0; c < nst; ++c) {
-      const int s = c % S;
-      const int b = c / kQaPromote;
-      const uint32_t buf = b & 1;
-      const bool first = c % kQaPromote == 0;
-      if (warp_flag(abort_flag)) break;
-      if (has_lr && first && b >= 2 &&
-          !warp_wait(smem_u32(&acc_empty[buf]), ((b >> 1) - 1) & 1, p.timeout_ns, 15)) {
-        *abort_flag = 1;
-        break;
-      }
-      if (!warp_wait(smem_u32(&quant[s]), (c / S) & 1, p.timeout_ns, 10)) {
-        *abort_flag = 1;
-        break;
-      }
-      if (has_lr) {
-        tc_fence_after();
-        const uint32_t d = tmem + RW * (1 + buf);
-        const int na = K - c * 128 >= 128 ? 2 : 1;
-        const uint32_t st = smem_base + s * stage_bytes;
-        for (int a = 0; a < na; ++a) {
-          const uint32_t l1a = st + a * katom_l1;
-          const uint32_t xa = st + l1_bytes + a * x_atom;
-          // second r-atom (A rows 64..127): loaded for r > 64, else the zero atom
-          const uint32_t lbo = r > 64 ? 8192u : zero_addr - l1a;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            e_mma_bf16(d, make_sdesc(l1a + kk * 2048, lbo, 1024, 2), make_sdesc(xa + kk * 32, 16, 1024, 2),
-                       idesc, (first && (a | kk) == 0) ? 0u : 1u);
-        }
-        e_commit(smem_u32(&freed[s]));
-        if (c % kQaPromote == kQaPromote - 1 || c == nst - 1) e_commit(smem_u32(&acc_full[buf]));
-      } else {
-        e_arrive(smem_u32(&freed[s]));
-      }
-    }
-    if (has_lr) e_commit(smem_u32(fin));
-  } else if (warp >= 18) {
-    // ------------------------------------------- fp32 running sum of T --
-    const int q = warp & 3;  // tensor-memory lane quadrant of this warp
-    const bool active = 32 * q < r;
-    const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-    const int j = 32 * q + lane;  // column of T held by this lane
-    for (int b = 0; has_lr && b < nblk; ++b) {
-      const uint32_t buf = b & 1;
-      if (!warp_wait(smem_u32(&acc_full[buf]), (b >> 1) & 1, p.timeout_ns, 16)) {
-        *abort_flag = 1;
-        break;
-      }
-      tc_fence_after();
-      if (active) {
-        const bool last = b == nblk - 1;
-        for (int n0 = 0; n0 < rows; n0 += 16) {
-          uint32_t v[16], t[16];
-          tmem_ld_32x32b_x16(tmem + lane_base + RW * (1 + buf) + n0, v);
-          if (b > 0) tmem_ld_32x32b_x16(tmem + lane_base + n0, t);
-          tmem_ld_wait();
-          if (b > 0) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              v[i] = __float_as_uint(__fadd_rn(__uint_as_float(t[i]), __uint_as_float(v[i])));
-          }
-          if (!last) {
-            tmem_st_32x32b_x16(tmem + lane_base + n0, v);
-          } else if (j < r) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int m = row0 + n0 + i;
-              if (m < p.M) p.T[static_cast<size_t>(m) * r + j] = __float2bfloat16_rn(__uint_as_float(v[i]));
-            }
-          }
-        }
-        if (!last) tmem_st_wait();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[buf]));
-    }
-  } else {
-    // ------------------------------------------------------- quantisers --
-    const int team = warp >> 3;
-    const int g = warp & 7;  // the 16-column group of each stage this warp quantises
-    for (int c = team; c < nst; c += 2) {
-      const int s = c % S;
-      // warp-uniform outcome: the warp meets __syncwarp below together
-      const bool ok = !warp_flag(abort_flag) && warp_wait(smem_u32(&full[s]), (c / S) & 1, p.timeout_ns, 12);
+      const bool ok = !warp_flag(abort_flag) && warp_wait(smem_u32(&full[s]), ph, p.timeout_ns, 12);
       if (!ok) {
         *abort_flag = 1;
         break;
       }
-      const int k = c * 128;
-      const int ng = K - k >= 128 ? 8 : 4;  // groups per row in this stage
-      if (g < ng) {
-        uint8_t* stage = smem + s * stage_bytes;
-        const float4* lam = reinterpret_cast<const float4*>(stage + l1_bytes + x_bytes) + 4 * g;
-        const float4 l0 = lam[0], l1 = lam[1], l2 = lam[2], l3 = lam[3];
-        const int kg = k + 16 * g;
-        const int j0 = (g & 3) * 2;  // logical 16-byte chunk of the row
-        uint8_t* atom = stage + l1_bytes + (g >> 2) * x_atom;
-        for (int rr = lane; rr < rows; rr += 32) {
-          uint8_t* row = atom + rr * 128;
-          const int sw = rr & 7;  // 128-byte swizzle phase of the row
-          uint4 w0 = *reinterpret_cast<const uint4*>(row + ((j0 ^ sw) << 4));
-          uint4 w1 = *reinterpret_cast<const uint4*>(row + (((j0 + 1) ^ sw) << 4));
-          float v[16];
-          v[0] = __fmul_rn(bf16_lo(w0.x), l0.x);  v[1] = __fmul_rn(bf16_hi(w0.x), l0.y);
-          v[2] = __fmul_rn(bf16_lo(w0.y), l0.z);  v[3] = __fmul_rn(bf16_hi(w0.y), l0.w);
-          v[4] = __fmul_rn(bf16_lo(w0.z), l1.x);  v[5] = __fmul_rn(bf16_hi(w0.z), l1.y);
-          v[6] = __fmul_rn(bf16_lo(w0.w), l1.z);  v[7] = __fmul_rn(bf16_hi(w0.w), l1.w);
-          v[8] = __fmul_rn(bf16_lo(w1.x), l2.x);  v[9] = __fmul_rn(bf16_hi(w1.x), l2.y);
-          v[10] = __fmul_rn(bf16_lo(w1.y), l2.z); v[11] = __fmul_rn(bf16_hi(w1.y), l2.w);
-          v[12] = __fmul_rn(bf16_lo(w1.z), l3.x); v[13] = __fmul_rn(bf16_hi(w1.z), l3.y);
-          v[14] = __fmul_rn(bf16_lo(w1.w), l3.z); v[15] = __fmul_rn(bf16_hi(w1.w), l3.w);
-          uint32_t lo, hi;
-          const uint32_t sc = nvfp4_group(v, lo, hi);
+      const int k = c * xw;
+      const int kv = min(xw, K - k);      // columns of this stage inside K
+      uint8_t* stage = smem + s * p.stage_bytes;
+      // 1. quantise: items (group, 32-row block) warp, warp + 16, ..., two at a time
+      for (int it = warp; it < items; it += 2 * kQaWarps) {
+        int gi[2], rri[2];
+        bool ok2[2];
+        uint4 w0[2], w1[2];
+        float4 lm[2][4];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const int item = it + kQaWarps * t;
+          const int ii = item < items ? item : it;  // a duplicate of the first item is computed, not stored
+          gi[t] = ii & (gs - 1);
+          rri[t] = ((ii >> gs_log2) << 5) + lane;
+          ok2[t] = item < items && 16 * gi[t] < kv && rri[t] < rows;
+          const int rrc = rri[t] < rows ? rri[t] : 0;
+          rri[t] = rrc;
+          const uint8_t* row = stage + (gi[t] >> 2) * x_atom + rrc * 128;
+          const uint32_t sw = static_cast<uint32_t>(rrc & 7) << 4;
+          const uint32_t c0 = static_cast<uint32_t>((gi[t] & 3) * 2) << 4;
+          w0[t] = *reinterpret_cast<const uint4*>(row + (c0 ^ sw));
+          w1[t] = *reinterpret_cast<const uint4*>(row + ((c0 + 16u) ^ sw));
+          const float4* lam = reinterpret_cast<const float4*>(stage + x_bytes + l1_bytes) + 4 * gi[t];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) lm[t][e] = lam[e];
+        }
+        float v[2][16];
+        uint32_t sc[2], lo[2], hi[2];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          mul2_rn(v[t][0], v[t][1], bf16_lo(w0[t].x), bf16_hi(w0[t].x), lm[t][0].x, lm[t][0].y);
+          mul2_rn(v[t][2], v[t][3], bf16_lo(w0[t].y), bf16_hi(w0[t].y), lm[t][0].z, lm[t][0].w);
+          mul2_rn(v[t][4], v[t][5], bf16_lo(w0[t].z), bf16_hi(w0[t].z), lm[t][1].x, lm[t][1].y);
+          mul2_rn(v[t][6], v[t][7], bf16_lo(w0[t].w), bf16_hi(w0[t].w), lm[t][1].z, lm[t][1].w);
+          mul2_rn(v[t][8], v[t][9], bf16_lo(w1[t].x), bf16_hi(w1[t].x), lm[t][2].x, lm[t][2].y);
+          mul2_rn(v[t][10], v[t][11], bf16_lo(w1[t].y), bf16_hi(w1[t].y), lm[t][2].z, lm[t][2].w);
+          mul2_rn(v[t][12], v[t][13], bf16_lo(w1[t].z), bf16_hi(w1[t].z), lm[t][3].x, lm[t][3].y);
+          mul2_rn(v[t][14], v[t][15], bf16_lo(w1[t].w), bf16_hi(w1[t].w), lm[t][3].z, lm[t][3].w);
+        }
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          float a0 = fmaxf(fabsf(v[t][0]), fabsf(v[t][1])), a1 = fmaxf(fabsf(v[t][2]), fabsf(v[t][3]));
+          float a2 = fmaxf(fabsf(v[t][4]), fabsf(v[t][5])), a3 = fmaxf(fabsf(v[t][6]), fabsf(v[t][7]));
+          a0 = fmaxf(a0, fmaxf(fabsf(v[t][8]), fabsf(v[t][9])));
+          a1 = fmaxf(a1, fmaxf(fabsf(v[t][10]), fabsf(v[t][11])));
+          a2 = fmaxf(a2, fmaxf(fabsf(v[t][12]), fabsf(v[t][13])));
+          a3 = fmaxf(a3, fmaxf(fabsf(v[t][14]), fabsf(v[t][15])));
+          const float amax = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+          sc[t] = cvt_e4m3_satfinite(__fdiv_rn(amax, 6.0f));
+        }
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const float rcp = rcp_tab[sc[t]];
+          float pq[16];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) mul2_rn(pq[e], pq[e + 1], v[t][e], v[t][e + 1], rcp, rcp);
+          lo[t] = cvt_e2m1x8(pq);
+          hi[t] = cvt_e2m1x8(pq + 8);
+        }
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (!ok2[t]) continue;
+          const int rr = rri[t];
           if (has_lr) {
-            w0 = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-            w1 = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
-                            pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
-            *reinterpret_cast<uint4*>(row + ((j0 ^ sw) << 4)) = w0;
-            *reinterpret_cast<uint4*>(row + (((j0 + 1) ^ sw) << 4)) = w1;
+            uint8_t* row = stage + (gi[t] >> 2) * x_atom + rr * 128;
+            const uint32_t sw = static_cast<uint32_t>(rr & 7) << 4;
+            const uint32_t c0 = static_cast<uint32_t>((gi[t] & 3) * 2) << 4;
+            *reinterpret_cast<uint4*>(row + (c0 ^ sw)) =
+                make_uint4(pack_bf16x2(v[t][0], v[t][1]), pack_bf16x2(v[t][2], v[t][3]),
+                           pack_bf16x2(v[t][4], v[t][5]), pack_bf16x2(v[t][6], v[t][7]));
+            *reinterpret_cast<uint4*>(row + ((c0 + 16u) ^ sw)) =
+                make_uint4(pack_bf16x2(v[t][8], v[t][9]), pack_bf16x2(v[t][10], v[t][11]),
+                           pack_bf16x2(v[t][12], v[t][13]), pack_bf16x2(v[t][14], v[t][15]));
           }
           const int m = row0 + rr;
+          const int kg = k + 16 * gi[t];
           if (m < p.M)
             *reinterpret_cast<uint2*>(p.x_codes + static_cast<size_t>(m) * (K >> 1) + (kg >> 1)) =
-                make_uint2(lo, hi);
-          if (m < p.m_pad) p.x_scales[scale_byte_offset(m, kg >> 4, K)] = static_cast<uint8_t>(sc);
+                make_uint2(lo[t], hi[t]);
+          if (m < p.m_pad)
+            p.x_scales[(static_cast<size_t>(m >> 7) * static_cast<size_t>(K >> 6) + (kg >> 6)) * 512 +
+                       (m & 31) * 16 + ((m & 127) >> 5) * 4 + ((kg >> 4) & 3)] = static_cast<uint8_t>(sc[t]);
         }
       }
-      if (has_lr) fence_proxy_async_smem();
+      // 2. low-rank partial product of the stage
+      if (has_lr) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&xready[s]));
+        if (!warp_wait(smem_u32(&xready[s]), ph, p.timeout_ns, 15)) {
+          *abort_flag = 1;
+          break;
+        }
+        const uint32_t xs_u = smem_u32(stage);
+        const uint32_t l1_u = xs_u + x_bytes;
+        const int ksv = kv / 16;
+#pragma unroll
+        for (int i = 0; i < kQaMaxUnits; ++i) {
+          if (i >= nu) break;
+          float acc[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+          for (int ks = kp; ks < ksv; ks += wpu) {
+            const uint32_t ac = static_cast<uint32_t>((((ks & 3) << 1) | (mi >> 1)) ^ a_sw[i]) << 4;
+            uint32_t a[4], b[4];
+            ldsm_x4(xs_u + (ks >> 2) * x_atom + a_off[i] + ac, a[0], a[1], a[2], a[3]);
+            ldsm_x4_trans(l1_u + b_off[i] + ks * b_kstep, b[0], b[1], b[2], b[3]);
+            mma_bf16_16816(acc, a, b[0], b[1], acc);
+            mma_bf16_16816(acc + 4, a, b[2], b[3], acc + 4);
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) tot[i][e] = __fadd_rn(tot[i][e], acc[e]);
+        }
+        fence_proxy_async_smem();  // bf16(Xh) writes before the next TMA into the stage
+      }
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&quant[s]));
+      if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
+      // warp 0 refills the slot of the previous stage once every warp is done with it
+      if (warp == 0 && c >= 1 && c - 1 + S < nst) {
+        const int sp = s == 0 ? S - 1 : s - 1;
+        const uint32_t pp = s == 0 ? ph ^ 1u : ph;
+        if (!warp_wait(smem_u32(&empty[sp]), pp, p.timeout_ns, 11)) {
+          *abort_flag = 1;
+          break;
+        }
+        load_stage(c - 1 + S, sp);
+        ++issued;
+      }
+      if (++s == S) {
+        s = 0;
+        ph ^= 1u;
+      }
     }
+    if (warp == 0 && warp_flag(abort_flag))  // let this CTA's own copies land before it can exit
+      for (int c = issued > S ? issued - S : 0; c < issued; ++c)
+        warp_wait(smem_u32(&full[c % S]), (c / S) & 1, p.timeout_ns, 14);
     // scale-layout padding rows that no tile covers: zero scales
     const int covered = gridDim.x * rows;
     if (blockIdx.x == gridDim.x - 1 && covered < p.m_pad) {
       const int gk = K >> 4;
-      for (int i = tid; i < (p.m_pad - covered) * gk; i += kQaQuantWarps * 32)
+      for (int i = tid; i < (p.m_pad - covered) * gk; i += kQaWarps * 32)
         p.x_scales[scale_byte_offset(covered + i / gk, i % gk, K)] = 0;
     }
   }
 
   if (has_lr) {
-    // every MMA of this CTA (also after an abort) completes before the
-    // tensor memory is released
-    if (!mbar_wait(smem_u32(fin), 0, p.timeout_ns, 13)) *abort_flag = 1;
+    // T = bf16(sum of the warps' partials), summed in the order kp = 0, 1, ..
+    float* part = reinterpret_cast<float*>(smem);  // the ring is idle now
+    __syncthreads();
+    if (nu > 0 && kp > 0)
+#pragma unroll
+      for (int e = 0; e < 8; e += 4)
+        *reinterpret_cast<float4*>(part + (((kp - 1) * U + warp % U) * 32 + lane) * 8 + e) =
+            make_float4(tot[0][e], tot[0][e + 1], tot[0][e + 2], tot[0][e + 3]);
+    __syncthreads();
+    if (nu > 0 && kp == 0 && !*abort_flag) {
+      const int gq = lane >> 2, tq = lane & 3;
+#pragma unroll
+      for (int i = 0; i < kQaMaxUnits; ++i) {
+        if (i >= nu) break;
+        const int u = U >= kQaWarps ? warp + kQaWarps * i : warp % U;
+        float t8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t8[e] = tot[i][e];
+        for (int q = 1; q < wpu; ++q) {
+          const float* src = part + (((q - 1) * U + u) * 32 + lane) * 8;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t8[e] = __fadd_rn(t8[e], src[e]);
+        }
+        const int rb = u / nbr, nb = u % nbr;
+#pragma unroll
+        for (int jn = 0; jn < 2; ++jn) {
+          const int col = nb * 16 + jn * 8 + 2 * tq;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int m = row0 + rb * 16 + gq + 8 * h;
+            if (m < p.M)
+              *reinterpret_cast<uint32_t*>(p.T + static_cast<size_t>(m) * r + col) =
+                  pack_bf16x2(t8[4 * jn + 2 * h], t8[4 * jn + 2 * h + 1]);
+          }
+        }
+      }
+    }
   }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 17 && has_lr) tmem_dealloc(tmem, tmem_cols);
 }
 
 // ================================================== fused 4-bit linear ====
@@ -486,8 +556,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
                   const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_l2,
                   const __grid_constant__ CUtensorMap tm_y, const LinParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   float* bias_s = reinterpret_cast<float*>(smem + kLinStages * kLinStageBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kLinBarOffset);
   uint64_t* full = bars;                           // [S] even CTA: both CTAs' stage landed

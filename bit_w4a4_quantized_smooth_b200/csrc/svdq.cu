@@ -80,12 +80,18 @@ int sm_count() {
 }
 
 // Rows per activation tile: a multiple of 16 in [16, 128] such that the
-// tiles cover M in about one wave over the SMs (one CTA per SM).
-int choose_rows(int64_t M, int sms) {
+// tiles cover M in about one wave over the SMs (one CTA per SM), and such that
+// the 16 x 16 tiles of T number at most two per warp (rows x r <= 8192).
+int choose_rows(int64_t M, int sms, int64_t r) {
   int64_t rows = (M + sms - 1) / sms;
   rows = (rows + 15) / 16 * 16;
+  int64_t cap = svdq::kQaMaxRows;
+  if (r > 0) {
+    const int64_t by_units = (2 * 16 / (r / 16)) * 16;
+    if (by_units < cap) cap = by_units;
+  }
+  if (rows > cap) rows = cap;
   if (rows < 16) rows = 16;
-  if (rows > svdq::kQaMaxRows) rows = svdq::kQaMaxRows;
   return static_cast<int>(rows);
 }
 
@@ -135,7 +141,7 @@ int svdq_quantize_act(const void* X, const float* inv_lambda, const void* L1, in
 
   const int sms = sm_count();
   if (sms <= 0) return SVDQ_ERR_CUDA;
-  const int rows = choose_rows(M, sms);
+  const int rows = choose_rows(M, sms, r);
   CUtensorMap tm_x, tm_l1;
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
@@ -145,21 +151,25 @@ int svdq_quantize_act(const void* X, const float* inv_lambda, const void* L1, in
                        CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
   }
+  const int ri = static_cast<int>(r);
+  const int xw = svdq::qa_xw(rows, ri);
+  const int aw = svdq::qa_aw(ri);
   if (r > 0) {
-    // L1 [K][r]: boxes of 64 (r, zero-filled past r) x 64 (k) with 128-byte
-    // swizzle are the MN-major atoms of the A operand L1^T.
+    // L1 [K][r] in atoms of aw columns x xw rows (boxes of up to 256 rows); the swizzle width is the
+    // atom's row (32, 64 or 128 bytes); columns past r arrive as zeros
     const uint64_t dims[2] = {static_cast<uint64_t>(r), static_cast<uint64_t>(K)};
     const uint64_t strides[1] = {static_cast<uint64_t>(r) * 2};
-    const uint32_t box[2] = {64, 64};
-    int rc = make_tmap(&tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L1, dims, strides, box,
-                       CU_TENSOR_MAP_SWIZZLE_128B);
+    const uint32_t box[2] = {static_cast<uint32_t>(aw), static_cast<uint32_t>(xw < 256 ? xw : 256)};
+    const CUtensorMapSwizzle sw = aw == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                           : (aw == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+    int rc = make_tmap(&tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L1, dims, strides, box, sw);
     if (rc) return rc;
   } else {
     std::memset(&tm_l1, 0, sizeof(tm_l1));
   }
 
-  const uint32_t stage_bytes = svdq::qa_stage_bytes(static_cast<int>(r), rows);
-  const uint32_t fixed = 1024 + svdq::qa_zero_bytes(static_cast<int>(r)) + svdq::kQaBarBytes;
+  const uint32_t stage_bytes = svdq::qa_stage_bytes(rows, ri);
+  const uint32_t fixed = 1024 + svdq::kQaBarBytes;
   int stages = static_cast<int>((svdq::kQaSmemLimit - fixed) / stage_bytes);
   if (stages > svdq::kQaMaxStages) stages = svdq::kQaMaxStages;
   if (stages < 2) return SVDQ_ERR_UNSUPPORTED_SHAPE;
@@ -170,10 +180,12 @@ int svdq_quantize_act(const void* X, const float* inv_lambda, const void* L1, in
   p.T = static_cast<__nv_bfloat16*>(T);
   p.M = static_cast<int>(M);
   p.K = static_cast<int>(K);
-  p.r = static_cast<int>(r);
+  p.r = ri;
   p.rows = rows;
-  p.stages = stages;
   p.m_pad = static_cast<int>((M + 127) / 128 * 128);
+  p.xw = xw;
+  p.aw = aw;
+  p.stages = stages;
   p.stage_bytes = stage_bytes;
   p.timeout_ns = wait_timeout_ns();
 
