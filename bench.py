@@ -49,7 +49,24 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
+    ap.add_argument("--once", choices=["quantize_act", "linear", "pack_residual"],
+                    help="no timing: three launches of one kernel on the workload (for profilers)")
     return ap.parse_args()
+
+
+# DRAM bytes (read + write) of one linear_kernel launch on flux_qkv from an
+# ncu capture (profiles/linear_kernel_flux_qkv.md; `bench.py --once linear`,
+# L2-warm).  Reported only while the kernel sources are the ones captured.
+LINEAR_TRAFFIC_CAPTURE = {"workload": "flux_qkv", "bytes": 24844032 + 30347008, "sources_sha256": "b6598c8ce4f2a03a"}
+
+
+def kernel_sources_sha():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("kernels.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "bit_w4a4_quantized_smooth_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 # ----------------------------------------------------------------- peaks ---
@@ -182,10 +199,15 @@ def oracle_sample(X_bits, inv, L1_bits, L2_bits, R, bias_bits, M, K, N, r, targe
         oracle.linear_rows(xc, xs, T, rc, rs, L2_bits, bias_bits, rows, K, N, r, np.arange(rows))
         return time.perf_counter() - t0
 
-    rows = 4
+    # grow the sample until it takes about target_s (small samples leave most
+    # OpenMP threads idle, so one probe underestimates the rate)
+    rows = min(M, 2 * oracle.num_threads())
     t = run(rows)
-    rows = int(max(4, min(M, rows * target_s / max(t, 1e-3))))
-    t = run(rows)
+    for _ in range(4):
+        if t >= 0.6 * target_s or rows >= M:
+            break
+        rows = int(max(rows + 1, min(M, rows * 0.9 * target_s / max(t, 1e-3))))
+        t = run(rows)
     return layer_flops(rows, K, N, r) / t / 1e12, rows, t, oracle.num_threads()
 
 
@@ -357,7 +379,11 @@ def run_ours(args, rank, world, local_rank):
             "peak": round(fp4_peak, 1),
             "unit": "TFLOP/s",
             "frac": round(achieved / fp4_peak, 4),
-            "traffic": None,
+            "traffic": (LINEAR_TRAFFIC_CAPTURE["bytes"]
+                        if args.workload == LINEAR_TRAFFIC_CAPTURE["workload"]
+                        and kernel_sources_sha() == LINEAR_TRAFFIC_CAPTURE["sources_sha256"] else None),
+            "traffic_note": "DRAM bytes of one launch from an ncu capture with L2 warm "
+                            "(bench.py --once linear); null when the kernel changed since",
             "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 4 (FP4/bf16 dense ratio)",
         },
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
@@ -379,6 +405,8 @@ def main():
         return 0
     import torch
     import torch.distributed as dist
+    if args.once:
+        return run_once(args)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -400,6 +428,32 @@ def main():
     finally:
         if world > 1:
             dist.destroy_process_group()
+    return 0
+
+
+def run_once(args):
+    """Three launches of one kernel on the workload, no timing, no L2 flush:
+    the command that profiler captures of a single kernel run."""
+    import torch
+    import bit_w4a4_quantized_smooth_b200 as svdq
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    L = setup_layer(args.workload, device)
+    M, K, N, r = L["M"], L["K"], L["N"], L["r"]
+    xc, xs, T = svdq.quantize_act(L["X"], L["inv"], L["L1"])
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    for _ in range(3):
+        if args.once == "quantize_act":
+            svdq.quantize_act(L["X"], L["inv"], L["L1"], x_codes=xc, x_scales=xs, T=T)
+        elif args.once == "linear":
+            svdq.linear(xc, xs, T, L["rc"], L["rs"], L["L2"], L["bias"], M, K, N, Y=Y)
+        else:
+            svdq.pack_residual(L["R"], r_codes=L["rc"], r_scales=L["rs"])
+    torch.cuda.synchronize()
+    st, where = svdq.sync_status()
+    if st != 0:
+        raise RuntimeError(f"kernel wait expired (id {where})")
+    print(json.dumps({"once": args.once, "workload": args.workload, "M": M, "K": K, "N": N, "r": r}))
     return 0
 
 
