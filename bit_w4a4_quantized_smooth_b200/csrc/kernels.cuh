@@ -2,7 +2,8 @@
 //
 //   pack_residual_kernel   R fp32 [K][N] -> NVFP4 codes [N][K/2] + tiled scales
 //   quantize_act_kernel    X bf16 [M][K] -> Xh = X * inv_lambda -> NVFP4 codes
-//                          and scales, and T = bf16(bf16(Xh) L1) on tcgen05
+//                          and scales, and T = bf16(bf16(Xh) L1) on warp-level
+//                          tensor-core MMAs from the same read of X
 //   linear_kernel          Y = deq(x) deq(R)^T + T L2 + bias on tcgen05:
 //                          block-scaled FP4 MMAs and the rank-r bf16 MMAs
 //                          accumulate into one fp32 tensor-memory tile.
