@@ -185,6 +185,25 @@ def linear_bytes(M, K, N, r):
     return 2 * M * K + N * K // 2 + N * K // 16 + 2 * K * r + 2 * r * N + 2 * M * N + 2 * N
 
 
+# ------------------------------------------------------ across ranks ---
+
+def max_over_ranks(x, device=None):
+    """The largest value of `x` over all ranks (x itself without a process
+    group): every multi-GPU number is the slowest rank's device time."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_step, steps_per_rank, world, max_ms):
+    """Every rank's work over the slowest rank's time (weak scaling)."""
+    return world * flops_per_step * steps_per_rank / (max_ms * 1e-3) / 1e12
+
+
 # -------------------------------------------------------- oracle (CPU) ---
 
 def oracle_sample(X_bits, inv, L1_bits, L2_bits, R, bias_bits, M, K, N, r, target_s):
@@ -272,18 +291,14 @@ def run_ours(args, rank, world, local_rank):
     qa_ms = [e[0].elapsed_time(e[1]) for e in ev]
     lin_ms = [e[1].elapsed_time(e[2]) for e in ev]
     step_ms = [a + b for a, b in zip(qa_ms, lin_ms)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), device)
     st, where = svdq.sync_status()
     if st != 0:
         raise RuntimeError(f"kernel wait expired in the timed region (id {where})")
 
     flops = layer_flops(M, K, N, r)
     ms_per_step = total_ms / args.steps
-    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+    value = whole_job_tflops(flops, args.steps, world, total_ms)
 
     # ---- per-kernel figures (this rank) ----
     qa_us = 1e3 * statistics.mean(qa_ms)
@@ -335,12 +350,8 @@ def run_ours(args, rank, world, local_rank):
         if i >= max(3, args.warmup):
             e2e.append((a, b))
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * flops * len(e2e) / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e), device)
+    e2e_value = whole_job_tflops(flops, len(e2e), world, e2e_ms)
 
     peaks = load_peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16

@@ -1,0 +1,71 @@
+"""The N > 1 path of bench.py on CPU: two gloo ranks (127.0.0.1).
+
+The layer is one GPU's work, so N GPUs run N replicas with no collective on
+the data path; the only cross-rank step is the timing: the slowest rank's
+time, and the whole job's work over it.
+"""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        local_ms = 10.0 + 5.0 * rank           # rank 1 is the slow one
+        slowest = bench.max_over_ranks(local_ms)
+        value = bench.whole_job_tflops(2.0e12, 4, world, slowest)
+        out[rank] = (slowest, value)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_whole_job_value_two_gloo_ranks():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    assert set(res) == {0, 1}
+    for rank in range(world):
+        slowest, value = res[rank]
+        assert slowest == 15.0                       # both ranks see the max
+        # 2 ranks x 4 steps x 2e12 flops over 15 ms
+        assert value == pytest.approx(2 * 4 * 2.0e12 / 15e-3 / 1e12)
+
+
+def test_single_process_needs_no_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(12.5) == 12.5
+    assert bench.whole_job_tflops(1e12, 10, 1, 100.0) == pytest.approx(100.0)
+
+
+def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
+    """Under torchrun only rank 0 runs and prints the reference line."""
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--gpus", "2"])
+    called = []
+    monkeypatch.setattr(bench, "run_reference", lambda args: called.append(1) or {})
+    assert bench.main() == 0
+    assert called == [] and capsys.readouterr().out == ""
