@@ -57,15 +57,21 @@ def parse_args():
 # DRAM bytes (read + write) of one linear_kernel launch on flux_qkv from an
 # ncu capture (profiles/linear_kernel_flux_qkv.md; `bench.py --once linear`,
 # L2-warm).  Reported only while the kernel sources are the ones captured.
-LINEAR_TRAFFIC_CAPTURE = {"workload": "flux_qkv", "bytes": 24844032 + 30347008, "sources_sha256": "a0cf3113ef1b40a2"}
+LINEAR_TRAFFIC_CAPTURE = {"workload": "flux_qkv", "bytes": 24844032 + 30347008, "sources_sha256": "49de90e47fe1ec0e"}
 
 
 def kernel_sources_sha():
+    """Hash of the linear kernel's source (its section of kernels.cuh) and of
+    the PTX helpers it is built from."""
     import hashlib
-    h = hashlib.sha256()
-    for f in ("kernels.cuh", "ptx.cuh"):
-        with open(os.path.join(ROOT, "bit_w4a4_quantized_smooth_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+    csrc = os.path.join(ROOT, "bit_w4a4_quantized_smooth_b200", "csrc")
+    with open(os.path.join(csrc, "kernels.cuh"), encoding="utf-8") as fh:
+        text = fh.read()
+    i = text.index("fused 4-bit linear ====")
+    j = text.index("bounded-wait self test ====")
+    h = hashlib.sha256(text[i:j].encode("utf-8"))
+    with open(os.path.join(csrc, "ptx.cuh"), "rb") as fh:
+        h.update(fh.read())
     return h.hexdigest()[:16]
 
 

@@ -279,7 +279,32 @@ __global__ void __launch_bounds__(kQaThreads, 1)
   }
   {
     const int gs_log2 = 31 - __clz(gs);
-    const int items = gs * ((rows + 31) >> 5);  // (group, 32-row block) pairs per stage
+    const int items = gs * ((rows + 31) >> 5);  // (group, 32-row block) pairs per stage, <= 32
+    // This warp's items are warp and warp + 16 in every stage (items <= 32),
+    // so their offsets are fixed: per stage only the column base moves.
+    int q_g[2];
+    bool q_row[2], q_code[2], q_scale[2];
+    uint32_t q_s0[2], q_s1[2];      // shared offsets of the item's two 16-byte chunks
+    size_t q_code_base[2], q_scale_base[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int item = warp + kQaWarps * t;
+      const int ii = item < items ? item : warp;  // a duplicate is computed, not stored
+      q_g[t] = ii & (gs - 1);
+      const int rr = ((ii >> gs_log2) << 5) + lane;
+      q_row[t] = item < items && rr < rows;
+      const int rrc = rr < rows ? rr : 0;
+      const uint32_t sw = static_cast<uint32_t>(rrc & 7) << 4;
+      const uint32_t c0 = static_cast<uint32_t>((q_g[t] & 3) * 2) << 4;
+      q_s0[t] = (q_g[t] >> 2) * x_atom + rrc * 128 + (c0 ^ sw);
+      q_s1[t] = (q_g[t] >> 2) * x_atom + rrc * 128 + ((c0 + 16u) ^ sw);
+      const int m = row0 + rrc;
+      q_code[t] = q_row[t] && m < p.M;
+      q_scale[t] = q_row[t] && m < p.m_pad;
+      q_code_base[t] = static_cast<size_t>(m) * static_cast<size_t>(K >> 1) + 8 * q_g[t];
+      q_scale_base[t] = static_cast<size_t>(m >> 7) * static_cast<size_t>(K >> 6) * 512 + (m & 31) * 16 +
+                        ((m & 127) >> 5) * 4 + (q_g[t] >> 2) * 512 + (q_g[t] & 3);
+    }
     const int mi = lane >> 3;            // ldmatrix: matrix this lane addresses
     // reciprocals of the 127 finite E4M3 scale values (0 for the zero scale)
     if (warp < 4) {
@@ -314,29 +339,17 @@ __global__ void __launch_bounds__(kQaThreads, 1)
       const int k = c * xw;
       const int kv = min(xw, K - k);      // columns of this stage inside K
       uint8_t* stage = smem + s * p.stage_bytes;
-      // 1. quantise: items (group, 32-row block) warp, warp + 16, ..., two at a time
-      for (int it = warp; it < items; it += 2 * kQaWarps) {
-        int gi[2], rri[2];
-        bool ok2[2];
+      // 1. quantise this warp's two items (independent chains, interleaved)
+      {
         uint4 w0[2], w1[2];
         float4 lm[2][4];
+        const float4* lam = reinterpret_cast<const float4*>(stage + x_bytes + l1_bytes);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          const int item = it + kQaWarps * t;
-          const int ii = item < items ? item : it;  // a duplicate of the first item is computed, not stored
-          gi[t] = ii & (gs - 1);
-          rri[t] = ((ii >> gs_log2) << 5) + lane;
-          ok2[t] = item < items && 16 * gi[t] < kv && rri[t] < rows;
-          const int rrc = rri[t] < rows ? rri[t] : 0;
-          rri[t] = rrc;
-          const uint8_t* row = stage + (gi[t] >> 2) * x_atom + rrc * 128;
-          const uint32_t sw = static_cast<uint32_t>(rrc & 7) << 4;
-          const uint32_t c0 = static_cast<uint32_t>((gi[t] & 3) * 2) << 4;
-          w0[t] = *reinterpret_cast<const uint4*>(row + (c0 ^ sw));
-          w1[t] = *reinterpret_cast<const uint4*>(row + ((c0 + 16u) ^ sw));
-          const float4* lam = reinterpret_cast<const float4*>(stage + x_bytes + l1_bytes) + 4 * gi[t];
+          w0[t] = *reinterpret_cast<const uint4*>(stage + q_s0[t]);
+          w1[t] = *reinterpret_cast<const uint4*>(stage + q_s1[t]);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) lm[t][e] = lam[e];
+          for (int e = 0; e < 4; ++e) lm[t][e] = lam[4 * q_g[t] + e];
         }
         float v[2][16];
         uint32_t sc[2], lo[2], hi[2];
@@ -371,29 +384,21 @@ __global__ void __launch_bounds__(kQaThreads, 1)
           lo[t] = cvt_e2m1x8(pq);
           hi[t] = cvt_e2m1x8(pq + 8);
         }
+        const size_t code_k = static_cast<size_t>(k >> 1);
+        const size_t scale_k = static_cast<size_t>(k >> 6) * 512;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          if (!ok2[t]) continue;
-          const int rr = rri[t];
+          if (!q_row[t] || 16 * q_g[t] >= kv) continue;
           if (has_lr) {
-            uint8_t* row = stage + (gi[t] >> 2) * x_atom + rr * 128;
-            const uint32_t sw = static_cast<uint32_t>(rr & 7) << 4;
-            const uint32_t c0 = static_cast<uint32_t>((gi[t] & 3) * 2) << 4;
-            *reinterpret_cast<uint4*>(row + (c0 ^ sw)) =
+            *reinterpret_cast<uint4*>(stage + q_s0[t]) =
                 make_uint4(pack_bf16x2(v[t][0], v[t][1]), pack_bf16x2(v[t][2], v[t][3]),
                            pack_bf16x2(v[t][4], v[t][5]), pack_bf16x2(v[t][6], v[t][7]));
-            *reinterpret_cast<uint4*>(row + ((c0 + 16u) ^ sw)) =
+            *reinterpret_cast<uint4*>(stage + q_s1[t]) =
                 make_uint4(pack_bf16x2(v[t][8], v[t][9]), pack_bf16x2(v[t][10], v[t][11]),
                            pack_bf16x2(v[t][12], v[t][13]), pack_bf16x2(v[t][14], v[t][15]));
           }
-          const int m = row0 + rr;
-          const int kg = k + 16 * gi[t];
-          if (m < p.M)
-            *reinterpret_cast<uint2*>(p.x_codes + static_cast<size_t>(m) * (K >> 1) + (kg >> 1)) =
-                make_uint2(lo[t], hi[t]);
-          if (m < p.m_pad)
-            p.x_scales[(static_cast<size_t>(m >> 7) * static_cast<size_t>(K >> 6) + (kg >> 6)) * 512 +
-                       (m & 31) * 16 + ((m & 127) >> 5) * 4 + ((kg >> 4) & 3)] = static_cast<uint8_t>(sc[t]);
+          if (q_code[t]) *reinterpret_cast<uint2*>(p.x_codes + q_code_base[t] + code_k) = make_uint2(lo[t], hi[t]);
+          if (q_scale[t]) p.x_scales[q_scale_base[t] + scale_k] = static_cast<uint8_t>(sc[t]);
         }
       }
       // 2. low-rank partial product of the stage
