@@ -339,25 +339,58 @@ def run_ours(args, rank, world, local_rank):
     pack_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in pk)
 
     # ---- end to end through the public API with host buffers ----
+    # A serving loop's schedule: three streams (host->device copy of X, the
+    # layer, device->host copy of Y) with double-buffered X and Y on the
+    # device, so that step i's copies overlap steps i-1 and i+1.  Every step
+    # still copies its own X in from pinned memory and its own Y out.  No L2
+    # flush inside this region: each step streams 113 MB of fresh X and Y
+    # through L2, with the weights a working set above L2's 126 MB.
     X_host = torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True)
     X_host.copy_(X)
-    Y_host = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
-    X_dev = torch.empty_like(X)
-    e2e = []
-    for i in range(max(3, args.warmup) + args.steps):
-        flush_l2()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        X_dev.copy_(X_host, non_blocking=True)
-        svdq.quantize_act(X_dev, inv, L1, x_codes=xc, x_scales=xs, T=T, stream=stream)
-        svdq.linear(xc, xs, T, rc, rs, L2, bias, M, K, N, Y=Y, stream=stream)
-        Y_host.copy_(Y, non_blocking=True)
-        b.record(stream)
-        if i >= max(3, args.warmup):
-            e2e.append((a, b))
+    Y_host = [torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
+    X_dev = [torch.empty_like(X) for _ in range(2)]
+    Y_dev = [torch.empty_like(Y) for _ in range(2)]
+    s_in = torch.cuda.Stream(device)
+    s_out = torch.cuda.Stream(device)
+    ev_in = [torch.cuda.Event() for _ in range(2)]    # X_dev[b] holds this step's X
+    ev_used = [torch.cuda.Event() for _ in range(2)]  # the layer is done with X_dev[b], Y_dev[b] written
+    ev_out = [torch.cuda.Event() for _ in range(2)]   # Y_dev[b] copied to the host
+
+    def run_e2e(nsteps):
+        for i in range(nsteps):
+            b = i & 1
+            if i >= 2:
+                s_in.wait_event(ev_used[b])
+            with torch.cuda.stream(s_in):
+                X_dev[b].copy_(X_host, non_blocking=True)
+            ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])
+            svdq.quantize_act(X_dev[b], inv, L1, x_codes=xc, x_scales=xs, T=T, stream=stream)
+            svdq.linear(xc, xs, T, rc, rs, L2, bias, M, K, N, Y=Y_dev[b], stream=stream)
+            ev_used[b].record(stream)
+            s_out.wait_event(ev_used[b])
+            with torch.cuda.stream(s_out):
+                Y_host[b].copy_(Y_dev[b], non_blocking=True)
+            ev_out[b].record(s_out)
+
+    run_e2e(max(3, args.warmup))
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e), device)
-    e2e_value = whole_job_tflops(flops, len(e2e), world, e2e_ms)
+    if world > 1:
+        dist.barrier()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_last_out = torch.cuda.Event()
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    s_in.wait_event(t_start)
+    run_e2e(args.steps)
+    t_last_out.record(s_out)
+    stream.wait_event(t_last_out)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(t_start.elapsed_time(t_end), device)
+    e2e_value = whole_job_tflops(flops, args.steps, world, e2e_ms)
 
     peaks = load_peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
@@ -404,7 +437,9 @@ def run_ours(args, rank, world, local_rank):
             "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 4 (FP4/bf16 dense ratio)",
         },
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
-                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
+                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
+                "ms_per_step": round(e2e_ms / args.steps, 4),
+                "schedule": "copy-in, layer and copy-out streams, double-buffered X and Y"},
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
     }
