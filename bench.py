@@ -57,7 +57,7 @@ def parse_args():
 # DRAM bytes (read + write) of one linear_kernel launch on flux_qkv from an
 # ncu capture (profiles/linear_kernel_flux_qkv.md; `bench.py --once linear`,
 # L2-warm).  Reported only while the kernel sources are the ones captured.
-LINEAR_TRAFFIC_CAPTURE = {"workload": "flux_qkv", "bytes": 24844032 + 30347008, "sources_sha256": "49de90e47fe1ec0e"}
+LINEAR_TRAFFIC_CAPTURE = {"workload": "flux_qkv", "bytes": 24844032 + 30347008, "sources_sha256": "f995a861848ff4cb"}
 
 
 def kernel_sources_sha():

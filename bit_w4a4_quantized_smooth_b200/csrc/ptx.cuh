@@ -1,6 +1,7 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers with bounded waits, TMA
-// (tensor and bulk copies), tcgen05 (TMEM allocation, MMA, copies, loads),
-// clusters and the NVFP4 conversion instructions.
+// (tensor and bulk copies, stores), tcgen05 across a CTA pair (TMEM
+// allocation, MMAs, scale copies, loads), warp-level MMAs, clusters and the
+// NVFP4 conversion instructions.
 #pragma once
 
 #include <cstdint>
@@ -36,11 +37,6 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
@@ -83,33 +79,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
 }
 
 // ------------------------------------------------------------------- TMA --
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int x,
-                                            int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(tmap), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint32_t bar, int x,
-                                            int y, int z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-      "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(bar)
-      : "memory");
-}
-
-// Untiled bulk copy global -> shared (16-byte aligned, size multiple of 16).
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
@@ -122,20 +91,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // --------------------------------------------------------------- tcgen05 --
-__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
-               "r"(ncols)
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
 
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -145,72 +100,8 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// Arrive on an mbarrier once all prior tcgen05 async ops of this thread finish.
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
-}
-
-// D (tmem) (+)= A (smem desc) x B (smem desc), bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                         uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// D (tmem) (+)= (A * SFA) x (B * SFB): FP4 E2M1 operands, UE4M3 scale per
-// 16 elements along K (scale factors read from tmem).
-__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
-      "p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
-}
-
-// Copy 32 rows x 128 bits from shared memory into tmem, replicated into the
-// four 32-lane quadrants.
-__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
-}
-
-// 32 lanes x 32 bit, 16 consecutive columns: thread t writes lane (base + t).
-__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t* v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_st_wait() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// 32 lanes x 32 bit, 16 consecutive columns: thread t gets lane (base + t).
-__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* v) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-        "=r"(v[14]), "=r"(v[15])
-      : "r"(taddr));
 }
 
 // 32 lanes x 32 bit, 32 consecutive columns: thread t gets lane (base + t).
@@ -247,16 +138,6 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uin
 }
 
 // ----------------------------------------------------- CTA-pair (2-SM) --
-// TMA load into this CTA's shared memory whose completion bytes go to the
-// mbarrier at `bar_cluster` (a shared::cluster address, possibly the peer's).
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, uint32_t bar_cluster,
-                                                 int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(tmap), "r"(x), "r"(y), "r"(bar_cluster)
-      : "memory");
-}
 
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
@@ -271,40 +152,6 @@ __device__ __forceinline__ void tmem_relinquish_pair() {
 __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
-}
-
-// MMAs across the CTA pair (issued by the even CTA): A rows split by CTA,
-// B columns split by CTA, D rows in each CTA's own tensor memory.
-__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                              uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                              uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                              uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
-      "p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
-}
-
-// Arrive once on the mbarrier at the same shared-memory offset in both CTAs
-// of the pair when all prior tcgen05 ops of this thread are complete.
-__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(bar),
-      "h"(static_cast<uint16_t>(3))
-      : "memory");
 }
 
 // Arrive on an mbarrier given by its shared::cluster address (release at
@@ -344,14 +191,6 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
   }
 }
 
-// 32 lanes x 32 bit, 8 consecutive columns.
-__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t* v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-      : "memory");
-}
-
 // ------------------------------------------------- warp-wide issue (elect) --
 // Issue loops run with the whole warp converged and let elect.sync pick the
 // single lane that executes the instruction: this keeps the loop's values on
@@ -366,16 +205,6 @@ __device__ __forceinline__ void e_arrive_expect_tx(uint32_t bar, uint32_t bytes)
                : "memory");
 }
 
-__device__ __forceinline__ void e_arrive(uint32_t bar) {
-  asm volatile(SVDQ_ELECT_BEGIN "@e mbarrier.arrive.shared::cta.b64 _, [%0];" SVDQ_ELECT_END ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void e_arrive_cluster(uint32_t bar_cluster) {
-  asm volatile(SVDQ_ELECT_BEGIN "@e mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" SVDQ_ELECT_END ::"r"(
-                   bar_cluster)
-               : "memory");
-}
-
 __device__ __forceinline__ void e_tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int x, int y) {
   asm volatile(SVDQ_ELECT_BEGIN
                "@e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
@@ -384,14 +213,8 @@ __device__ __forceinline__ void e_tma_load_2d(uint32_t dst, const void* tmap, ui
                : "memory");
 }
 
-__device__ __forceinline__ void e_tma_load_3d(uint32_t dst, const void* tmap, uint32_t bar, int x, int y, int z) {
-  asm volatile(SVDQ_ELECT_BEGIN
-               "@e cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-               " [%0], [%1, {%2, %3, %4}], [%5];" SVDQ_ELECT_END ::"r"(dst),
-               "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(bar)
-               : "memory");
-}
-
+// TMA load into this CTA's shared memory whose completion bytes go to the
+// mbarrier at `bar_cluster` (a shared::cluster address, possibly the peer's).
 __device__ __forceinline__ void e_tma_load_2d_pair(uint32_t dst, const void* tmap, uint32_t bar_cluster, int x,
                                                    int y) {
   asm volatile(SVDQ_ELECT_BEGIN
@@ -401,6 +224,7 @@ __device__ __forceinline__ void e_tma_load_2d_pair(uint32_t dst, const void* tma
                : "memory");
 }
 
+// Untiled bulk copy global -> shared (16-byte aligned, size multiple of 16).
 __device__ __forceinline__ void e_bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(SVDQ_ELECT_BEGIN
                "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" SVDQ_ELECT_END ::
@@ -409,14 +233,8 @@ __device__ __forceinline__ void e_bulk_load(uint32_t dst, const void* src, uint3
                : "memory");
 }
 
-__device__ __forceinline__ void e_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                           uint32_t accumulate) {
-  asm volatile(SVDQ_ELECT_BEGIN ".reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-               "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;" SVDQ_ELECT_END ::"r"(d_tmem),
-               "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-               : "memory");
-}
-
+// MMAs across the CTA pair (issued by the even CTA): A rows split by CTA,
+// B columns split by CTA, D rows in each CTA's own tensor memory.
 __device__ __forceinline__ void e_mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                                 uint32_t accumulate) {
   asm volatile(SVDQ_ELECT_BEGIN ".reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
@@ -425,6 +243,8 @@ __device__ __forceinline__ void e_mma_bf16_pair(uint32_t d_tmem, uint64_t adesc,
                : "memory");
 }
 
+// D (tmem) (+)= (A * SFA) x (B * SFB): FP4 E2M1 operands, UE4M3 scale per
+// 16 elements along K (scale factors read from tmem).
 __device__ __forceinline__ void e_mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                                 uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
   asm volatile(SVDQ_ELECT_BEGIN ".reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
@@ -434,12 +254,8 @@ __device__ __forceinline__ void e_mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc,
                : "memory");
 }
 
-__device__ __forceinline__ void e_commit(uint32_t bar) {
-  asm volatile(SVDQ_ELECT_BEGIN "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" SVDQ_ELECT_END ::
-                   "r"(bar)
-               : "memory");
-}
-
+// Arrive once on the mbarrier at the same shared-memory offset in both CTAs
+// of the pair when all prior tcgen05 ops of this thread are complete.
 __device__ __forceinline__ void e_commit_pair_both(uint32_t bar) {
   asm volatile(SVDQ_ELECT_BEGIN
                "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
@@ -545,7 +361,6 @@ __device__ __forceinline__ uint32_t map_shared_rank(uint32_t saddr, uint32_t ran
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
-
 
 // ------------------------------------------------------- NVFP4 convert --
 // fp32 -> E4M3 (round to nearest even, saturating); returns the byte.
