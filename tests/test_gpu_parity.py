@@ -3,8 +3,8 @@
 * packed codes and scales: bit-exact (integer work decided in fp32 on both
   sides: the same RN_f32 products and quotients, then RNE to E4M3/E2M1);
 * T = bf16(bf16(Xh) L1): within one bf16 ulp of the oracle's fp64 sum
-  rounded once (fp32 tensor-core accumulation may flip a rounding), and at
-  least 98 % of the elements bit-identical;
+  rounded once (fp32 accumulation may flip a rounding), and at least 99.9 %
+  of the elements bit-identical (at most 2 flips in tiny cases);
 * Y: relative Frobenius error <= 2e-3 against the oracle's fp64 Y, where
   the output rounding to bf16 alone contributes about 1e-3.
 """
@@ -52,11 +52,11 @@ def _lib():
 def check_T(T_gpu_bits, T_or_bits):
     a = bf16_bits_to_f64(T_gpu_bits)
     b = bf16_bits_to_f64(T_or_bits)
-    same = np.mean(T_gpu_bits == T_or_bits)
+    flips = int(np.count_nonzero(T_gpu_bits != T_or_bits))
     ulp = np.spacing(np.abs(b).astype(np.float32)).astype(np.float64) * 65536.0  # bf16 ulp
     tiny = 1e-30 + 1e-6 * np.abs(b).max()
     assert np.all(np.abs(a - b) <= ulp + tiny), np.abs(a - b).max()
-    assert same >= 0.98, same
+    assert flips <= max(2, 0.001 * T_gpu_bits.size), (flips, T_gpu_bits.size)
 
 
 def rel_fro(Y, ref):
