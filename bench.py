@@ -51,6 +51,8 @@ def parse_args():
                     help="target CPU time of the oracle sample")
     ap.add_argument("--once", choices=["quantize_act", "linear", "pack_residual"],
                     help="no timing: three launches of one kernel on the workload (for profilers)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="the K = N = 3072 sweep over M and rank: one JSON line per point")
     return ap.parse_args()
 
 
@@ -436,6 +438,11 @@ def run_ours(args, rank, world, local_rank):
                             "(bench.py --once linear); null when the kernel changed since",
             "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 4 (FP4/bf16 dense ratio)",
         },
+        "spec_sheet": {"fp4_tflops": SPEC_FP4_TFLOPS, "hbm_gbs": SPEC_HBM_GBS,
+                       "linear_frac": round(achieved / SPEC_FP4_TFLOPS, 4),
+                       "layer_roofline_frac": round(max(flops / (SPEC_FP4_TFLOPS * 1e12),
+                                                        linear_bytes(M, K, N, r) / (SPEC_HBM_GBS * 1e9))
+                                                    * 1e6 / (1e3 * ms_per_step), 4)},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
                 "ms_per_step": round(e2e_ms / args.steps, 4),
@@ -459,6 +466,8 @@ def main():
     import torch.distributed as dist
     if args.once:
         return run_once(args)
+    if args.sweep:
+        return run_sweep(args)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -506,6 +515,80 @@ def run_once(args):
     if st != 0:
         raise RuntimeError(f"kernel wait expired (id {where})")
     print(json.dumps({"once": args.once, "workload": args.workload, "M": M, "K": K, "N": N, "r": r}))
+    return 0
+
+
+SPEC_FP4_TFLOPS = 9000.0   # B200 dense FP4 (the spec sheet's 18 PF is 2:4 sparse)
+SPEC_HBM_GBS = 8000.0
+
+
+def run_sweep(args):
+    """The memory-bound sweep at K = N = 3072: every M in SWEEP_M and rank in
+    SWEEP_R, one W and one smoothing calibration (4608 rows) for all points,
+    the SVD taken once per rank, X the leading M rows of one draw.  Each point
+    times the layer (quantize_act + linear) with L2 flushed before every rep
+    and reports TFLOP/s and the layer's algorithmic bytes per second."""
+    import torch
+    import bit_w4a4_quantized_smooth_b200 as svdq
+    from bit_w4a4_quantized_smooth_b200 import prep
+    from svdq_inputs import make_layer_inputs
+    from svdq_inputs.workloads import SWEEP_M, SWEEP_R
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    li = make_layer_inputs("sweep_3072", M=max(SWEEP_M), r=max(SWEEP_R), cal_rows=4608)
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+
+    X, W, Xcal = bf16(li.X), bf16(li.W), bf16(li.Xcal)
+    bias = None if li.bias is None else bf16(li.bias)
+    lam, inv = prep.smoothing(Xcal, W)
+    K, N = li.K, li.N
+    peaks = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    flush_rd = torch.zeros(L2_FLUSH_BYTES // 8, dtype=torch.float32, device=device)
+    reps = max(5, min(args.steps, 20))
+    for r in SWEEP_R:
+        L1, L2, R = prep.lowrank(W, lam, r)
+        rc, rs = svdq.pack_residual(R)
+        del R
+        for M in SWEEP_M:
+            Xm = X[:M]
+            xc, xs, T = svdq.quantize_act(Xm, inv, L1)
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+            for _ in range(3):
+                svdq.quantize_act(Xm, inv, L1, x_codes=xc, x_scales=xs, T=T)
+                svdq.linear(xc, xs, T, rc, rs, L2, bias, M, K, N, Y=Y)
+            ev = []
+            for _ in range(reps):
+                flush.zero_()
+                flush_rd.sum()
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                e[0].record()
+                svdq.quantize_act(Xm, inv, L1, x_codes=xc, x_scales=xs, T=T)
+                e[1].record()
+                svdq.linear(xc, xs, T, rc, rs, L2, bias, M, K, N, Y=Y)
+                e[2].record()
+                ev.append(e)
+            torch.cuda.synchronize()
+            st, where = svdq.sync_status()
+            if st != 0:
+                raise RuntimeError(f"kernel wait expired (id {where})")
+            qa_us = 1e3 * statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+            lin_us = 1e3 * statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+            us = qa_us + lin_us
+            flops = layer_flops(M, K, N, r)
+            nbytes = linear_bytes(M, K, N, r)
+            roof_us = max(flops / (fp4_peak * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9)) * 1e6
+            print(json.dumps({
+                "sweep": "K=N=3072", "M": M, "rank": r, "us_per_layer": round(us, 2),
+                "quantize_act_us": round(qa_us, 2), "linear_us": round(lin_us, 2),
+                "tflops": round(flops / (us * 1e-6) / 1e12, 2),
+                "algorithmic_gbs": round(nbytes / (us * 1e-6) / 1e9, 1),
+                "bound": "tensor" if flops / (fp4_peak * 1e12) > nbytes / (peaks["hbm_gbs"] * 1e9) else "hbm",
+                "roofline_frac": round(roof_us / us, 4), "reps": reps,
+                "l2": "flushed before every rep"}), flush=True)
     return 0
 
 
