@@ -116,21 +116,24 @@ __global__ void __launch_bounds__(kPackThreads) pack_residual_kernel(const float
 
 // ============================================ activation quantise + T =====
 // One CTA per tile of `rows` consecutive rows of X (rows in {16, 32, .., 128},
-// chosen so that the tiles fill the SMs once), over all of K: no split of the
+// chosen so that the tiles fill the SMs once, and with rows x r <= 8192 so
+// that a warp holds at most two 16 x 16 tiles of T), over all of K: no split of the
 // reduction, hence no partial sums to combine across CTAs.  512 threads, all
 // computing; warp 0 also issues the TMA loads (warp-wide, elect.sync), one
 // stage behind the consumers, so that four warps per sub-core keep up to 128
 // registers each.
 //
 // A ring stage holds xw = 512, 256 or 128 columns of the tile (the widest
-// that still leaves a few stages of shared memory): the X atoms (64 columns, K-major, 128-byte swizzle), the matching xw
-// rows of L1 as atoms of aw = r (16 or 32) or 64 columns (32/64/128-byte
-// swizzle, columns past r arrive as zeros) and the inv_lambda values.
+// that still leaves a few stages of shared memory): the X atoms (64 columns,
+// K-major, 128-byte swizzle), the matching xw rows of L1 as atoms of aw = r
+// (16 or 32) or 64 columns (32/64/128-byte swizzle, columns past r arrive as
+// zeros) and the inv_lambda values.
 // Per stage every compute warp
-//   1. quantises 16-column groups of 32 rows (one row per lane), two at a time
-//      so that each thread has two independent dependency chains in flight:
-//      codes and scale to global memory, bf16(Xh) back into the X atom in
-//      place;
+//   1. quantises its two items, (16-column group, 32-row block) number w and
+//      w + 16 of the stage (one row per lane; the same items every stage, so
+//      their offsets are computed once), interleaved so that each thread has
+//      two independent dependency chains in flight: codes and scale to global
+//      memory, bf16(Xh) back into the X atom in place;
 //   2. after all 16 warps have written bf16(Xh) (an mbarrier), adds its share
 //      of Xh L1 with warp-level tensor-core MMAs (m16n8k16, bf16 in, fp32 out;
 //      fragments by ldmatrix from the swizzled atoms) into a stage partial,
@@ -140,7 +143,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_residual_kernel(const float
 // to 128 (measured), and one issuing thread per CTA would need K / 16 of them
 // in series, 8 us at K = 3072.  Spread over 16 warps and the four sub-core
 // tensor units it hides under the HBM stream.  Folding each stage's partial
-// (K <= 256) into fp32 keeps long K as accurate as an fp32 sum (tensor-core
+// (K <= 512) into fp32 keeps long K as accurate as an fp32 sum (tensor-core
 // accumulation over thousands of terms drifts by several bf16 ulps).
 // T tiles (16 x 16) are split over the warps; when there are fewer than 16,
 // several warps share a tile over disjoint k-steps and the partials are summed
