@@ -49,3 +49,16 @@ def lowrank(W: torch.Tensor, lam: torch.Tensor, r: int):
     L2 = V.T.contiguous().to(torch.bfloat16)
     R = (Wh - L1.double() @ L2.double()).float()
     return L1.contiguous(), L2.contiguous(), R.contiguous()
+
+
+def attach_lora(L1, L2, lam: torch.Tensor, A: torch.Tensor, B: torch.Tensor):
+    """Join a LoRA adapter A bf16 [K][ra], B bf16 [ra][N] to the low-rank
+    branch without re-quantising the residual (chattools.cn
+    "SVDQuant的主要功能", item LoRA集成): with Xh = X diag(lambda)^-1,
+    Xh [L1 | diag(lambda) A] [L2 ; B] = Xh L1 L2 + X A B.
+    -> (L1' bf16 [K][r+ra], L2' bf16 [r+ra][N]); lambda A is one fp32
+    product per element, rounded once to bf16."""
+    LA = (lam.float()[:, None] * A.float()).to(torch.bfloat16)
+    L1n = LA if L1 is None else torch.cat([L1, LA], dim=1)
+    L2n = B if L2 is None else torch.cat([L2, B], dim=0)
+    return L1n.contiguous(), L2n.contiguous()

@@ -78,6 +78,7 @@ def lib() -> ctypes.CDLL:
             ("oracle_sym_eig_top", [_P, _I64, _I64, _P, _P]),
             ("oracle_svd_top", [_P, _I64, _I64, _I64, _P, _P, _P]),
             ("oracle_lowrank", [_P, _P, _I64, _I64, _I64, _P, _P, _P, _P]),
+            ("oracle_attach_lora", [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P]),
             ("oracle_quantize_act", [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P]),
             ("oracle_dequant", [_P, _P, _I64, _I64, _P]),
             ("oracle_linear_rows", [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _I64, _P]),
@@ -213,6 +214,25 @@ def lowrank(W: np.ndarray, lam: np.ndarray, r: int):
     _check(lib().oracle_lowrank(_ptr(W), _ptr(lam), K, N, r, _ptr(L1), _ptr(L2), _ptr(R), _ptr(s)),
            "lowrank")
     return L1, L2, R, s
+
+
+def attach_lora(L1: Optional[np.ndarray], L2: Optional[np.ndarray], lam: np.ndarray, A: np.ndarray,
+                B: np.ndarray):
+    """LoRA A [K][ra], B [ra][N] (bf16 bits) joined to the low-rank branch:
+    -> (L1' [K][r+ra], L2' [r+ra][N]) bf16 bits; the residual is unchanged."""
+    A = np.ascontiguousarray(A, dtype=np.uint16)
+    B = np.ascontiguousarray(B, dtype=np.uint16)
+    lam = np.ascontiguousarray(lam, dtype=np.float32)
+    K, ra = A.shape
+    N = B.shape[1]
+    r = 0 if L1 is None else L1.shape[1]
+    L1c = np.zeros((K, 0), np.uint16) if L1 is None else np.ascontiguousarray(L1, dtype=np.uint16)
+    L2c = np.zeros((0, N), np.uint16) if L2 is None else np.ascontiguousarray(L2, dtype=np.uint16)
+    L1o = np.zeros((K, r + ra), dtype=np.uint16)
+    L2o = np.zeros((r + ra, N), dtype=np.uint16)
+    _check(lib().oracle_attach_lora(_ptr(L1c), _ptr(L2c), _ptr(lam), _ptr(A), _ptr(B), K, N, r, ra,
+                                    _ptr(L1o), _ptr(L2o)), "attach_lora")
+    return L1o, L2o
 
 
 def quantize_act(X: np.ndarray, inv_lambda: np.ndarray, L1: Optional[np.ndarray], r: int):

@@ -561,6 +561,32 @@ int oracle_lowrank(const uint16_t* W, const float* lambda, int64_t K, int64_t N,
   return 0;
 }
 
+// LoRA adapter joined to the low-rank branch without re-quantising the
+// residual (chattools.cn "SVDQuant的主要功能", item LoRA集成; the abstract: an
+// adapter needs no re-quantisation).  With Xh = X diag(lambda)^-1,
+//   Xh [L1 | diag(lambda) A] [L2 ; B] = Xh L1 L2 + X A B,
+// so L1' = [L1 | bf16(RN_f32(lambda_k a_kj))], L2' = [L2 ; B] and R stays.
+//   L1 [K][r], A [K][ra], L2 [r][N], B [ra][N] bf16 bits -> L1o [K][r+ra],
+//   L2o [r+ra][N].
+int oracle_attach_lora(const uint16_t* L1, const uint16_t* L2, const float* lambda, const uint16_t* A,
+                       const uint16_t* B, int64_t K, int64_t N, int64_t r, int64_t ra, uint16_t* L1o,
+                       uint16_t* L2o) {
+  if (K <= 0 || N <= 0 || r < 0 || ra <= 0) return 1;
+  const int64_t ro = r + ra;
+  for (int64_t k = 0; k < K; ++k) {
+    for (int64_t j = 0; j < r; ++j) L1o[k * ro + j] = L1[k * r + j];
+    for (int64_t j = 0; j < ra; ++j) {
+      const float prod = lambda[k] * bf16_to_f32(A[k * ra + j]);  // one fp32 rounding
+      L1o[k * ro + r + j] = bf16_from_f64(static_cast<double>(prod));
+    }
+  }
+  for (int64_t j = 0; j < r; ++j)
+    for (int64_t n = 0; n < N; ++n) L2o[j * N + n] = L2[j * N + n];
+  for (int64_t j = 0; j < ra; ++j)
+    for (int64_t n = 0; n < N; ++n) L2o[(r + j) * N + n] = B[j * N + n];
+  return 0;
+}
+
 // Activation step (quantise + low-rank down-projection), rows of X:
 //   Xh  = RN_f32(X * inv_lambda)             per element
 //   (x_codes, x_scales) = NVFP4(Xh) by groups of 16 along K
