@@ -38,7 +38,8 @@ def _rank_main(rank, world, port, out):
 def test_max_over_ranks_and_whole_job_value_two_gloo_ranks():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    # spawn, not fork: the test process may already run OpenMP threads
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
