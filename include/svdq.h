@@ -31,6 +31,10 @@
  *  - Argument errors are detected on the host before anything is launched
  *    and returned as a status; no call aborts or exits.
  *  - Inputs must be finite; NaN or Inf gives unspecified codes.
+ *  - LoRA adapters (chattools.cn, item "LoRA集成": no re-quantisation) need
+ *    no call of their own: an adapter A [K][ra], B [ra][N] joins the
+ *    low-rank branch as L1' = [L1 | bf16(lambda A)], L2' = [L2 ; B] (rank
+ *    r + ra <= 128), since Xh diag(lambda) A = X A; R stays as packed.
  *
  * Packed NVFP4 layout (codes and scales)
  * --------------------------------------
