@@ -207,6 +207,19 @@ def max_over_ranks(x, device=None):
     return float(t.item())
 
 
+def step_stats(ms):
+    """Median, p10 and p90 of per-step times in µs (the single value when
+    only one step ran)."""
+    us = sorted(1e3 * float(x) for x in ms)
+    if not us:
+        return None
+    if len(us) == 1:
+        return {"median_us": round(us[0], 2), "p10_us": round(us[0], 2), "p90_us": round(us[0], 2)}
+    dec = statistics.quantiles(us, n=10, method="inclusive")
+    return {"median_us": round(statistics.median(us), 2), "p10_us": round(dec[0], 2),
+            "p90_us": round(dec[-1], 2)}
+
+
 def whole_job_tflops(flops_per_step, steps_per_rank, world, max_ms):
     """Every rank's work over the slowest rank's time (weak scaling)."""
     return world * flops_per_step * steps_per_rank / (max_ms * 1e-3) / 1e12
@@ -415,6 +428,7 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic",
         "config": dict(workload_desc(args.workload, M, K, N, r), parallelism=f"replicas{world}"),
         "us_per_layer": round(1e3 * ms_per_step, 2),
+        "step_us": step_stats(step_ms),
         "quantize_act_us": round(qa_us, 2),
         "linear_us": round(lin_us, 2),
         "linear_r0_us": round(lin_r0_us, 2),

@@ -93,3 +93,14 @@ def test_reference_arm_prints_the_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert "workload" in d["config"]
+
+
+def test_step_stats():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.step_stats([]) is None
+    one = bench.step_stats([0.1])
+    assert one == {"median_us": 100.0, "p10_us": 100.0, "p90_us": 100.0}
+    st = bench.step_stats([0.1 + 0.001 * i for i in range(50)])   # 100 .. 149 µs
+    assert st["median_us"] == pytest.approx(124.5)
+    assert 100.0 <= st["p10_us"] < st["median_us"] < st["p90_us"] <= 149.0
