@@ -7,8 +7,8 @@ then svdq_linear (block-scaled FP4 GEMM + low-rank up-projection + bias).
 The residual packer runs once per weight; it is timed separately and
 reported beside the step (pack_residual_us).
 
-Default workload: the FLUX.1-shaped attention QKV projection, M = 4608
-tokens (4096 image + 512 text), K = 3072, N = 9216, rank 32, synthetic data.
+Default workload: the FLUX.1-shaped MLP up-projection, M = 4608 tokens
+(4096 image + 512 text), K = 3072, N = 12288, rank 32, synthetic data.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -45,7 +45,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="flux_qkv")
+    ap.add_argument("--workload", default="flux_mlp_up")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
@@ -56,10 +56,12 @@ def parse_args():
     return ap.parse_args()
 
 
-# DRAM bytes (read + write) of one linear_kernel launch on flux_qkv from an
-# ncu capture (profiles/linear_kernel_flux_qkv.md; `bench.py --once linear`,
-# L2-warm).  Reported only while the kernel sources are the ones captured.
-LINEAR_TRAFFIC_CAPTURE = {"workload": "flux_qkv", "bytes": 24844032 + 30347008, "sources_sha256": "f995a861848ff4cb"}
+# DRAM bytes (read + write) of one linear_kernel launch from an ncu capture of
+# `bench.py --once linear --workload <name>` (L2-warm), per workload.  A figure
+# is reported only while the kernel sources hash to the captured ones.
+LINEAR_TRAFFIC_CAPTURES = {
+    "flux_qkv": {"bytes": 24844032 + 30347008, "sources_sha256": "f995a861848ff4cb"},
+}
 
 
 def kernel_sources_sha():
@@ -75,6 +77,13 @@ def kernel_sources_sha():
     with open(os.path.join(csrc, "ptx.cuh"), "rb") as fh:
         h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+def linear_traffic(workload):
+    cap = LINEAR_TRAFFIC_CAPTURES.get(workload)
+    if cap is None or kernel_sources_sha() != cap["sources_sha256"]:
+        return None
+    return cap["bytes"]
 
 
 # ----------------------------------------------------------------- peaks ---
@@ -358,8 +367,9 @@ def run_ours(args, rank, world, local_rank):
     # layer, device->host copy of Y) with double-buffered X and Y on the
     # device, so that step i's copies overlap steps i-1 and i+1.  Every step
     # still copies its own X in from pinned memory and its own Y out.  No L2
-    # flush inside this region: each step streams 113 MB of fresh X and Y
-    # through L2, with the weights a working set above L2's 126 MB.
+    # flush inside this region: each step streams its fresh X and Y through
+    # L2, while the packed weights (a few tens of MB) may stay L2-resident
+    # from one step to the next, as they would in a serving loop.
     X_host = torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True)
     X_host.copy_(X)
     Y_host = [torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
@@ -409,7 +419,9 @@ def run_ours(args, rank, world, local_rank):
 
     peaks = load_peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
-    achieved = flops / (lin_us * 1e-6) / 1e12
+    # the linear kernel's own work: the FP4 product and the rank-r up-projection
+    lin_flops = 2.0 * M * N * K + 2.0 * M * N * r
+    achieved = lin_flops / (lin_us * 1e-6) / 1e12
     qa_bytes = 2 * M * K + M * K // 2 + M * K // 16 + 2 * M * r + 2 * K * r + 4 * K
     layer_roof_us = max(flops / (fp4_peak * 1e12), linear_bytes(M, K, N, r) / (peaks["hbm_gbs"] * 1e9)) * 1e6
 
@@ -445,9 +457,7 @@ def run_ours(args, rank, world, local_rank):
             "peak": round(fp4_peak, 1),
             "unit": "TFLOP/s",
             "frac": round(achieved / fp4_peak, 4),
-            "traffic": (LINEAR_TRAFFIC_CAPTURE["bytes"]
-                        if args.workload == LINEAR_TRAFFIC_CAPTURE["workload"]
-                        and kernel_sources_sha() == LINEAR_TRAFFIC_CAPTURE["sources_sha256"] else None),
+            "traffic": linear_traffic(args.workload),
             "traffic_note": "DRAM bytes of one launch from an ncu capture with L2 warm "
                             "(bench.py --once linear); null when the kernel changed since",
             "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 4 (FP4/bf16 dense ratio)",

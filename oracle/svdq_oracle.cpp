@@ -18,8 +18,8 @@
 //     (NVFP4: E2M1 values, one unsigned E4M3 scale per 16 consecutive
 //     elements along K, scale = amax / 6);
 //   * Y = Xh L1 L2 + Q(Xh) Q(R) (+ bias).
-// Readings where the pages are silent (rounding order, layouts, zero groups)
-// are listed in the design doc and restated beside each function below.
+// Where the pages are silent (rounding order, layouts, zero groups) the
+// reading taken is stated beside each function below.
 //
 // Arithmetic: fp64 everywhere except where a rounding step is part of the
 // encoding contract (fp32 products/quotients of the quantiser, the bf16 and

@@ -31,6 +31,8 @@ from .workloads import (  # noqa: F401
     LayerInputs,
     make_layer_inputs,
     make_activation,
+    make_lora,
+    make_stack_layer_inputs,
     make_weight,
     stack_layer_shapes,
 )

@@ -125,7 +125,17 @@ CONFIGS = {
                           lo=1.0, hi=1.0, w="gauss", q=0, bias=None),
     "sweep_3072": dict(config=4, M=4608, K=3072, N=3072, r=32, x="outlier", n_out=31, lo=20.0,
                        hi=100.0, w="planted", q=8, bias=0.01),
+    # the two shapes of the synthetic DiT stack that no other workload has
+    # (a single-stream block's fused input and output projections), with the
+    # stack's rank-32 LoRA adapter; seeds are those of stack layers 76 and 77
+    "dit_single_in": dict(config=5, layer=76, M=4608, K=3072, N=21504, r=32, x="outlier", n_out=31,
+                          lo=20.0, hi=100.0, w="gauss", q=0, bias=None, lora=32),
+    "dit_single_out": dict(config=5, layer=77, M=4608, K=15360, N=3072, r=32, x="gelu", n_out=0,
+                           lo=1.0, hi=1.0, w="gauss", q=0, bias=None, lora=32),
 }
+
+# LoRA adapter of every DiT-stack layer: rank 32, A ~ N(0, 0.01), B ~ N(0, 0.01)
+STACK_LORA_RANK = 32
 
 SWEEP_M = (1, 16, 64, 256, 1024, 4096, 16384)
 SWEEP_R = (16, 32, 64, 128)
@@ -158,7 +168,30 @@ def make_layer_inputs(name: str, M: Optional[int] = None, K: Optional[int] = Non
         Xcal = make_activation(seed, _S_XCAL, cal_rows, K, c["x"], n_out, c["lo"], c["hi"])
     W = make_weight(seed, K, N, c["w"], c["q"])
     bias = make_bias(seed, N, c["bias"])
-    return LayerInputs(name=name, M=M, K=K, N=N, r=r, X=X, W=W, bias=bias, Xcal=Xcal)
+    A = B = None
+    if c.get("lora"):
+        A, B = make_lora(seed, K, N, c["lora"])
+    return LayerInputs(name=name, M=M, K=K, N=N, r=r, X=X, W=W, bias=bias, Xcal=Xcal,
+                       lora_A=A, lora_B=B)
+
+
+def make_stack_layer_inputs(layer: int, M: int = 4608, with_x: bool = True) -> LayerInputs:
+    """Inputs of layer ``layer`` (0..151) of the synthetic 12B DiT stack:
+    W ~ N(0, 0.02) [K][N], no bias, a rank-32 LoRA adapter, and (unless
+    ``with_x`` is false) M activation rows, hidden-state-like (outlier
+    channels) for the 3072-wide inputs and GELU for the MLP/fused outputs."""
+    K, N, kind = stack_layer_shapes()[layer]
+    seed = config_seed(5, layer)
+    if with_x:
+        n_out = 31 if kind == "outlier" else 0
+        lo, hi = (20.0, 100.0) if kind == "outlier" else (1.0, 1.0)
+        X = make_activation(seed, _S_X, M, K, kind, n_out, lo, hi)
+    else:
+        X = np.zeros((0, K), dtype=np.uint16)
+    W = make_weight(seed, K, N, "gauss", 0)
+    A, B = make_lora(seed, K, N, STACK_LORA_RANK)
+    return LayerInputs(name=f"dit_stack[{layer}]", M=M, K=K, N=N, r=32, X=X, W=W, bias=None, Xcal=X,
+                       lora_A=A, lora_B=B)
 
 
 def stack_layer_shapes():

@@ -35,12 +35,19 @@ class Prepared:
 
 @functools.lru_cache(maxsize=8)
 def prepare(workload: str, M=None, K=None, N=None, r=None, cal_rows=None) -> Prepared:
+    """The oracle's preparation of a workload.  A workload that carries a
+    LoRA adapter gets it joined to the low-rank branch (the oracle's
+    attach_lora), so that ``r`` is then the SVD rank plus the adapter's."""
     li = make_layer_inputs(workload, M=M, K=K, N=N, r=r, cal_rows=cal_rows)
     lam, inv = oracle.smooth(li.Xcal, li.W)
     L1, L2, R, _ = oracle.lowrank(li.W, lam, li.r)
+    rank = li.r
     if li.r == 0:
         L1 = L2 = None
-    return Prepared(li.name, li.M, li.K, li.N, li.r, li.X, lam, inv, L1, L2, R, li.bias)
+    if li.lora_A is not None:
+        L1, L2 = oracle.attach_lora(L1, L2, lam, li.lora_A, li.lora_B)
+        rank += li.lora_A.shape[1]
+    return Prepared(li.name, li.M, li.K, li.N, rank, li.X, lam, inv, L1, L2, R, li.bias)
 
 
 def to_device(p: Prepared):

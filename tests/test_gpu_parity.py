@@ -20,14 +20,14 @@ pytestmark = pytest.mark.gpu
 Y_TOL = 2e-3
 
 # (workload, M, K, N, r): several tiles, ragged M / N / K tails, r = 0,
-# r = 128 (two low-rank stages), M = 1, an 8-CTA cluster (K = 2048)
+# r = 128 (two low-rank stages), M = 1, a long K with r = 48
 SMALL = [
     ("tiny", None, None, None, None),            # the full tiny layer 256 x 1024 x 1024, r 16
     ("flux_qkv", 200, 320, 272, 32),             # ragged M, N (one 128-row scale band) and K
     ("flux_mlp_up", 130, 256, 512, 0),           # no low-rank branch
     ("flux_mlp_down", 384, 512, 256, 128),       # GELU inputs, two low-rank stages
     ("flux_qkv", 1, 1024, 256, 64),              # one token
-    ("sweep_3072", 128, 2048, 256, 48),          # cluster of 8 along K, r = 48
+    ("sweep_3072", 128, 2048, 256, 48),          # K = 2048 (32 groups per row), r = 48
     ("flux_qkv", 300, 192, 528, 16),             # K = 3 chunks, N tail of 16 columns
     ("flux_qkv", 160, 384, 256, 96),             # r = 96: second r-atom of L1 partly past r
 ]
@@ -61,6 +61,34 @@ def check_T(T_gpu_bits, T_or_bits):
 
 def rel_fro(Y, ref):
     return float(np.linalg.norm(Y - ref) / np.linalg.norm(ref))
+
+
+def abs_terms(xc, xs, T, rc, rs, L2, bias, M, K, N, r, rows):
+    """E[i][n] = sum_k |deq x_ik deq R_nk| + sum_j |T_ij L2_jn| + |bias_n|,
+    the magnitude the fp32 accumulation error of Y[i][n] scales with."""
+    Xd = np.abs(oracle.dequant(xc, xs, M, K)[rows].astype(np.float64))
+    Rd = np.abs(oracle.dequant(rc, rs, N, K).astype(np.float64))
+    E = Xd @ Rd.T
+    if r:
+        E += np.abs(bf16_bits_to_f64(T)[rows]) @ np.abs(bf16_bits_to_f64(L2))
+    if bias is not None:
+        E += np.abs(bf16_bits_to_f64(bias))[None, :]
+    return E
+
+
+def check_Y_elementwise(Yg, ref, E, K, r):
+    """Every element within the output rounding plus an fp32 accumulation
+    term: Y = bf16(acc + bias) with acc an fp32 sum of K/64 block products
+    and r/16 low-rank products, so |Y - Y64| <= 1/2 ulp_bf16(max(|Y|, |Y64|))
+    + n_add 2^-23 E, with n_add = K/64 + r/16 + 2 additions each off by at
+    most one fp32 ulp of the running sum.  A dropped term on one column block
+    (a missing bias, a lost K block) exceeds this by orders of magnitude."""
+    big = np.maximum(np.abs(Yg), np.abs(ref)).astype(np.float32)
+    half_ulp = np.spacing(big).astype(np.float64) * 65536.0 / 2.0
+    n_add = K // 64 + (r + 15) // 16 + 2
+    bound = half_ulp + n_add * 2.0 ** -23 * E + 1e-30
+    excess = np.abs(Yg - ref) - bound
+    assert excess.max() <= 0, (float(excess.max()), np.unravel_index(int(np.argmax(excess)), excess.shape))
 
 
 @pytest.mark.parametrize("case", SMALL, ids=_ids)
@@ -106,9 +134,12 @@ def test_linear_on_oracle_operands(case):
     Y = svdq.linear(dev(oxc), dev(oxs), Tt, dev(orc), dev(ors), d["L2"], d["bias"], p.M, p.K, p.N)
     torch.cuda.synchronize()
     Yg = bf16_bits_to_f64(bf16_to_np_bits(Y))
-    ref = oracle.linear_rows(oxc, oxs, oT, orc, ors, p.L2, p.bias, p.M, p.K, p.N, p.r, np.arange(p.M))
+    rows = np.arange(p.M)
+    ref = oracle.linear_rows(oxc, oxs, oT, orc, ors, p.L2, p.bias, p.M, p.K, p.N, p.r, rows)
     err = rel_fro(Yg, ref)
     assert err <= Y_TOL, err
+    E = abs_terms(oxc, oxs, oT, orc, ors, p.L2, p.bias, p.M, p.K, p.N, p.r, rows)
+    check_Y_elementwise(Yg, ref, E, p.K, p.r)
     assert svdq.sync_status()[0] == 0
 
 
@@ -127,9 +158,12 @@ def test_layer_end_to_end(case):
     Yg = bf16_bits_to_f64(bf16_to_np_bits(Y))
     oxc, oxs, oT = oracle.quantize_act(p.X, p.inv, p.L1, p.r)
     orc, ors = oracle.pack_residual(p.R)
-    ref = oracle.linear_rows(oxc, oxs, oT, orc, ors, p.L2, p.bias, p.M, p.K, p.N, p.r, np.arange(p.M))
+    rows = np.arange(p.M)
+    ref = oracle.linear_rows(oxc, oxs, oT, orc, ors, p.L2, p.bias, p.M, p.K, p.N, p.r, rows)
     err = rel_fro(Yg, ref)
     assert err <= Y_TOL, err
+    E = abs_terms(oxc, oxs, oT, orc, ors, p.L2, p.bias, p.M, p.K, p.N, p.r, rows)
+    check_Y_elementwise(Yg, ref, E, p.K, p.r)
     assert svdq.sync_status()[0] == 0
 
 
@@ -202,6 +236,9 @@ def _layer_vs_oracle_rows(p, rows):
     # every sampled row on its own, so that no tile hides behind the average
     per_row = np.linalg.norm(Yg - ref, axis=1) / np.linalg.norm(ref, axis=1)
     assert per_row.max() <= 2 * Y_TOL, per_row.max()
+    # and every sampled element
+    E = abs_terms(oxc, oxs, oT, orc, ors, p.L2, p.bias, p.M, p.K, p.N, p.r, rows)
+    check_Y_elementwise(Yg, ref, E, p.K, p.r)
     return err
 
 
@@ -220,6 +257,10 @@ FULL = [
     # the sweep's smoothing is calibrated on one 4608-row draw for every M
     ("sweep_3072", 16384, None, None, 128, 4608),
     ("sweep_3072", 1, None, None, 16, 4608),
+    # the DiT stack's two shapes found nowhere else, each with the rank-32
+    # SVD branch joined to a rank-32 LoRA adapter (rank 64 through the kernels)
+    ("dit_single_in", None, None, None, None),
+    ("dit_single_out", None, None, None, None),
 ]
 
 
