@@ -65,17 +65,14 @@ LINEAR_TRAFFIC_CAPTURES = {
 
 
 def kernel_sources_sha():
-    """Hash of the linear kernel's source (its section of kernels.cuh) and of
-    the PTX helpers it is built from."""
+    """Hash of the linear kernel's sources: its header and the helpers it is
+    built from."""
     import hashlib
     csrc = os.path.join(ROOT, "bit_w4a4_quantized_smooth_b200", "csrc")
-    with open(os.path.join(csrc, "kernels.cuh"), encoding="utf-8") as fh:
-        text = fh.read()
-    i = text.index("fused 4-bit linear ====")
-    j = text.index("bounded-wait self test ====")
-    h = hashlib.sha256(text[i:j].encode("utf-8"))
-    with open(os.path.join(csrc, "ptx.cuh"), "rb") as fh:
-        h.update(fh.read())
+    h = hashlib.sha256()
+    for name in ("linear.cuh", "common.cuh", "ptx.cuh"):
+        with open(os.path.join(csrc, name), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()[:16]
 
 

@@ -10,6 +10,7 @@ binding raises if the library is missing.
 
 from .binding import (  # noqa: F401
     SvdqError,
+    attach_lora,
     lib_path,
     linear,
     load,
@@ -17,6 +18,8 @@ from .binding import (  # noqa: F401
     packed_sizes,
     quantize_act,
     selftest_wait_timeout,
+    set_linear_path,
+    set_wait_timeout,
     status_string,
     sync_status,
 )

@@ -51,13 +51,21 @@ def load() -> ctypes.CDLL:
         L.svdq_pack_residual.restype = ctypes.c_int
         L.svdq_pack_residual.argtypes = [_P, _I64, _I64, _P, _P, _P]
         L.svdq_quantize_act.restype = ctypes.c_int
-        L.svdq_quantize_act.argtypes = [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P]
+        L.svdq_quantize_act.argtypes = [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, ctypes.c_size_t, _P]
+        L.svdq_quantize_act_workspace.restype = ctypes.c_int
+        L.svdq_quantize_act_workspace.argtypes = [_I64, _I64, _I64, ctypes.POINTER(ctypes.c_size_t)]
         L.svdq_linear.restype = ctypes.c_int
         L.svdq_linear.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P]
         L.svdq_sync_status.restype = ctypes.c_int
         L.svdq_sync_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int)]
         L.svdq_selftest_wait_timeout.restype = ctypes.c_int
         L.svdq_selftest_wait_timeout.argtypes = [ctypes.c_uint64, _P]
+        L.svdq_set_wait_timeout.restype = ctypes.c_int
+        L.svdq_set_wait_timeout.argtypes = [ctypes.c_uint64]
+        L.svdq_attach_lora.restype = ctypes.c_int
+        L.svdq_attach_lora.argtypes = [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P]
+        L.svdq_set_linear_path.restype = ctypes.c_int
+        L.svdq_set_linear_path.argtypes = [ctypes.c_int]
         _lib = L
     return _lib
 
@@ -103,9 +111,36 @@ def pack_residual(R, r_codes=None, r_scales=None, stream=None):
     return r_codes, r_scales
 
 
-def quantize_act(X, inv_lambda, L1, x_codes=None, x_scales=None, T=None, stream=None):
+def quantize_act_workspace_bytes(M: int, K: int, r: int) -> int:
+    n = ctypes.c_size_t()
+    _check(load().svdq_quantize_act_workspace(M, K, r, ctypes.byref(n)), "svdq_quantize_act_workspace")
+    return n.value
+
+
+# Zero-filled scratch per (device, stream), grown on demand: the calls leave
+# its counters at zero, and calls on one stream never overlap.
+_workspaces = {}
+
+
+def workspace(nbytes: int, device, stream=None):
+    """A zero-initialised device buffer of at least `nbytes` bytes for calls
+    on `stream` (the current stream by default)."""
+    import torch
+    if nbytes == 0:
+        return None
+    key = (str(device), _stream(stream))
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
+def quantize_act(X, inv_lambda, L1, x_codes=None, x_scales=None, T=None, stream=None, workspace_buf=None):
     """X bf16 [M][K], inv_lambda fp32 [K], L1 bf16 [K][r] or None ->
-    (x_codes uint8 [M][K/2], x_scales uint8 tiled, T bf16 [M][r] or None)."""
+    (x_codes uint8 [M][K/2], x_scales uint8 tiled, T bf16 [M][r] or None).
+    The scratch the call needs comes from `workspace_buf` (zero-filled before
+    its first use) or from the binding's per-stream buffer."""
     import torch
     M, K = X.shape
     r = 0 if L1 is None else L1.shape[1]
@@ -116,8 +151,11 @@ def quantize_act(X, inv_lambda, L1, x_codes=None, x_scales=None, T=None, stream=
         x_scales = torch.empty(sb, dtype=torch.uint8, device=X.device)
     if T is None and r > 0:
         T = torch.empty((M, r), dtype=torch.bfloat16, device=X.device)
+    need = quantize_act_workspace_bytes(M, K, r)
+    ws = workspace_buf if workspace_buf is not None else workspace(need, X.device, stream)
     _check(load().svdq_quantize_act(_ptr(X), _ptr(inv_lambda), _ptr(L1), M, K, r, _ptr(x_codes),
-                                    _ptr(x_scales), _ptr(T), _stream(stream)), "svdq_quantize_act")
+                                    _ptr(x_scales), _ptr(T), _ptr(ws), 0 if ws is None else ws.numel(),
+                                    _stream(stream)), "svdq_quantize_act")
     return x_codes, x_scales, T
 
 
@@ -134,11 +172,41 @@ def linear(x_codes, x_scales, T, r_codes, r_scales, L2, bias, M: int, K: int, N:
     return Y
 
 
+def attach_lora(L1, L2, lam, A, B, L1_out=None, L2_out=None, stream=None):
+    """Join a LoRA adapter (A bf16 [K][ra], B bf16 [ra][N]) to the low-rank
+    branch (L1 [K][r], L2 [r][N], or None for r = 0) on the device ->
+    (L1' bf16 [K][r+ra], L2' bf16 [r+ra][N])."""
+    import torch
+    K, ra = A.shape
+    N = B.shape[1]
+    r = 0 if L1 is None else L1.shape[1]
+    if L1_out is None:
+        L1_out = torch.empty((K, r + ra), dtype=torch.bfloat16, device=A.device)
+    if L2_out is None:
+        L2_out = torch.empty((r + ra, N), dtype=torch.bfloat16, device=A.device)
+    _check(load().svdq_attach_lora(_ptr(L1), _ptr(L2), _ptr(lam), _ptr(A), _ptr(B), K, N, r, ra, _ptr(L1_out),
+                                   _ptr(L2_out), _stream(stream)), "svdq_attach_lora")
+    return L1_out, L2_out
+
+
 def sync_status(stream=None) -> Tuple[int, int]:
     """(status, wait id) recorded by the kernels since the last call."""
     where = ctypes.c_int(0)
     st = load().svdq_sync_status(_stream(stream), ctypes.byref(where))
     return st, where.value
+
+
+def set_wait_timeout(timeout_ns: int):
+    """Limit (ns) of every bounded wait in kernels launched from now on."""
+    _check(load().svdq_set_wait_timeout(timeout_ns), "svdq_set_wait_timeout")
+
+
+LINEAR_PATHS = {"auto": 0, "large": 1, "small": 2}
+
+
+def set_linear_path(path: str):
+    """Force svdq_linear's kernel: "auto" (by shape), "large" or "small"."""
+    _check(load().svdq_set_linear_path(LINEAR_PATHS[path]), "svdq_set_linear_path")
 
 
 def selftest_wait_timeout(timeout_ns: int, stream=None):

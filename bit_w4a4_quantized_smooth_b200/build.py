@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsvdq.so")
 SOURCES = [os.path.join(CSRC, "svdq.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("kernels.cuh", "ptx.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
     os.path.join(HERE, "..", "include", "svdq.h")]
 
 NVCC_FLAGS = [

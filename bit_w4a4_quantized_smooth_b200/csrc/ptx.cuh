@@ -137,6 +137,21 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uin
   return d;
 }
 
+// ------------------------------------------------------ single CTA (1-SM) --
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
 // ----------------------------------------------------- CTA-pair (2-SM) --
 
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
@@ -224,12 +239,68 @@ __device__ __forceinline__ void e_tma_load_2d_pair(uint32_t dst, const void* tma
                : "memory");
 }
 
+// Prefetch a 2-D box of a tensor into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void e_tma_prefetch_2d(const void* tmap, int x, int y) {
+  asm volatile(SVDQ_ELECT_BEGIN "@e cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" SVDQ_ELECT_END ::"l"(
+                   tmap),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 // Untiled bulk copy global -> shared (16-byte aligned, size multiple of 16).
 __device__ __forceinline__ void e_bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(SVDQ_ELECT_BEGIN
                "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" SVDQ_ELECT_END ::
                    "r"(dst),
                "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// One CTA's MMA: D (tmem) (+)= A x B, bf16 operands, fp32 accumulator.
+__device__ __forceinline__ void e_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(SVDQ_ELECT_BEGIN ".reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;" SVDQ_ELECT_END ::"r"(d_tmem),
+               "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+               : "memory");
+}
+
+// One CTA's block-scaled FP4 MMA (E2M1 operands, UE4M3 scale per 16 along K,
+// scale factors read from tmem).
+__device__ __forceinline__ void e_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(SVDQ_ELECT_BEGIN ".reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;" SVDQ_ELECT_END ::
+                   "r"(d_tmem),
+               "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+               : "memory");
+}
+
+// Arrive once on this CTA's mbarrier when all prior tcgen05 ops of this
+// thread are complete.
+__device__ __forceinline__ void e_commit(uint32_t bar) {
+  asm volatile(SVDQ_ELECT_BEGIN "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" SVDQ_ELECT_END ::
+                   "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void e_arrive(uint32_t bar) {
+  asm volatile(SVDQ_ELECT_BEGIN "@e mbarrier.arrive.shared::cta.b64 _, [%0];" SVDQ_ELECT_END ::"r"(bar) : "memory");
+}
+
+// Copy 32 rows x 128 bits from shared memory into tensor memory, replicated
+// into the four 32-lane quadrants (one CTA).
+__device__ __forceinline__ void e_tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile(SVDQ_ELECT_BEGIN "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" SVDQ_ELECT_END ::"r"(taddr),
+               "l"(sdesc)
+               : "memory");
+}
+
+__device__ __forceinline__ void e_tma_load_3d(uint32_t dst, const void* tmap, uint32_t bar, int x, int y, int z) {
+  asm volatile(SVDQ_ELECT_BEGIN
+               "@e cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+               " [%0], [%1, {%2, %3, %4}], [%5];" SVDQ_ELECT_END ::"r"(dst),
+               "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(bar)
                : "memory");
 }
 
@@ -262,6 +333,19 @@ __device__ __forceinline__ void e_commit_pair_both(uint32_t bar) {
                " [%0], %1;" SVDQ_ELECT_END ::"r"(bar),
                "h"(static_cast<uint16_t>(3))
                : "memory");
+}
+
+// Retire `bytes` expected transaction bytes of an mbarrier's current phase
+// as if they had arrived (one elected lane; no arrival is counted).
+__device__ __forceinline__ void e_mbar_complete_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile(SVDQ_ELECT_BEGIN "@e mbarrier.complete_tx.shared::cta.b64 [%0], %1;" SVDQ_ELECT_END ::"r"(bar),
+               "r"(bytes)
+               : "memory");
+}
+
+// Store a 32-bit value to a shared::cluster address (possibly the peer CTA's).
+__device__ __forceinline__ void st_dsmem_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
 // Warp-uniform bounded waits: every lane polls, lane 0's outcome decides for
@@ -303,6 +387,13 @@ __device__ __forceinline__ void e_tmem_cp_pair_32x128b_warpx4(uint32_t taddr, ui
 __device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int x, int y) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(tmap), "r"(src),
                "r"(x), "r"(y)
+               : "memory");
+}
+
+// Untiled bulk copy shared -> global (bulk-group completion; 16-byte aligned,
+// size a multiple of 16).
+__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
                : "memory");
 }
 
@@ -354,6 +445,31 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
+}
+
+// Four fp32 values from a shared::cluster address (possibly another CTA's).
+__device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
 }
 
 __device__ __forceinline__ uint32_t map_shared_rank(uint32_t saddr, uint32_t rank) {

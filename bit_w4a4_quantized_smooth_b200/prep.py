@@ -9,8 +9,10 @@ and the rest is the residual that the packer quantises to 4 bits.
     Wh = diag(lambda) W,  Wh ~ U_r S_r V_r^T  (top-r eigenpairs of the Gram matrix)
     L1 = bf16(U_r S_r), L2 = bf16(V_r^T), R = fp32(Wh - L1 L2)
 
-It uses torch's library linear algebra (matmul, eigh) in fp64 on the device:
-preparation is not part of the forward pass that the library's kernels run.
+It uses torch's library linear algebra (matmul, eigh, QR, SVD) in fp64 on the
+device: preparation is not part of the forward pass that the library's
+kernels run.  lowrank() takes the top-r eigenpairs of the Gram matrix;
+lowrank_randomized() a randomized subspace iteration for many layers at once.
 """
 
 from __future__ import annotations
@@ -47,6 +49,38 @@ def lowrank(W: torch.Tensor, lam: torch.Tensor, r: int):
         U = (Wh @ V) / torch.where(s > 0, s, torch.ones_like(s))
     L1 = (U * s).to(torch.bfloat16)
     L2 = V.T.contiguous().to(torch.bfloat16)
+    R = (Wh - L1.double() @ L2.double()).float()
+    return L1.contiguous(), L2.contiguous(), R.contiguous()
+
+
+def lowrank_randomized(W: torch.Tensor, lam: torch.Tensor, r: int, oversample: int = 16,
+                       power_iters: int = 2, seed: int = 0):
+    """The same factors as lowrank() from a randomized range finder instead
+    of a full eigendecomposition: Halko, Martinsson and Tropp, "Finding
+    structure with randomness" (SIAM Review 53, 2011), Algorithm 4.4
+    (randomized subspace iteration, re-orthonormalised after every product),
+    then the SVD of the small projected matrix.  fp64 on the device, a few
+    matmuls and QRs of width r + oversample: milliseconds where the Gram
+    eigendecomposition of a 3072-wide layer takes most of a second.  The
+    top-r subspace is approximate (exact on a rank-r matrix); R is still
+    exactly Wh - L1 L2 rounded to fp32, so the layer's reconstruction holds.
+    -> (L1 bf16 [K][r] or None, L2 bf16 [r][N] or None, R fp32 [K][N])."""
+    Wh = lam.double()[:, None] * W.double()
+    K, N = Wh.shape
+    if r == 0:
+        return None, None, Wh.float()
+    l = min(r + oversample, K, N)
+    gen = torch.Generator(device=Wh.device)
+    gen.manual_seed(seed)
+    omega = torch.randn((N, l), generator=gen, device=Wh.device, dtype=torch.float64)
+    Q, _ = torch.linalg.qr(Wh @ omega)
+    for _ in range(power_iters):
+        Z, _ = torch.linalg.qr(Wh.T @ Q)
+        Q, _ = torch.linalg.qr(Wh @ Z)
+    Ub, s, Vt = torch.linalg.svd(Q.T @ Wh, full_matrices=False)
+    U = Q @ Ub[:, :r]
+    L1 = (U * s[:r]).to(torch.bfloat16)
+    L2 = Vt[:r].contiguous().to(torch.bfloat16)
     R = (Wh - L1.double() @ L2.double()).float()
     return L1.contiguous(), L2.contiguous(), R.contiguous()
 

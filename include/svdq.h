@@ -21,11 +21,17 @@
  * Conventions shared by every call
  * --------------------------------
  *  - All tensors are dense, row-major, in DEVICE memory, allocated and owned
- *    by the caller.  The library allocates no memory and keeps no state
- *    besides a per-device status word (see svdq_sync_status).
+ *    by the caller.  The library allocates no device memory.  Its host-side
+ *    state is a cache of encoded TMA descriptors (a pure function of the
+ *    buffers' addresses and shapes, so reuse is always valid) and the
+ *    kernels' shared-memory limits set per device; on the device it keeps a
+ *    per-device status word (see svdq_sync_status).  All calls are safe to
+ *    make from several host threads.
  *  - bf16 tensors are passed as `const void*` / `void*` (IEEE bfloat16).
  *  - Every pointer must be 16-byte aligned.  K must be a multiple of 64,
- *    N a multiple of 16, r one of 0, 16, 32, ..., 128, M >= 1.
+ *    N a multiple of 16, r one of 0, 16, 32, ..., 128, M >= 1.  Sizes are
+ *    bounded by M, N <= 2^22 and K <= 2^20 (SVDQ_ERR_UNSUPPORTED_SHAPE
+ *    beyond), which keeps every grid dimension and index in range.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
  *    are asynchronous and stream-ordered; none synchronises.
  *  - Argument errors are detected on the host before anything is launched
@@ -73,7 +79,7 @@ const char* svdq_status_string(int status);
 /* Bytes of the packed buffers for `rows` vectors of length K:
  * codes_bytes = rows * K / 2, scales_bytes = ceil(rows / 128) * 128 * K / 16.
  * Host-only; K must be a multiple of 64. */
-int svdq_packed_sizes(int64_t rows, int64_t K, size_t* codes_bytes, size_t* scales_bytes);
+svdq_status svdq_packed_sizes(int64_t rows, int64_t K, size_t* codes_bytes, size_t* scales_bytes);
 
 /*
  * Residual packer, run once per weight (the 4-bit residual of the SVDQuant
@@ -84,8 +90,15 @@ int svdq_packed_sizes(int64_t rows, int64_t K, size_t* codes_bytes, size_t* scal
  *                                   channel n, groups of 16 along K
  *   r_scales uint8, svdq_packed_sizes(N, K) bytes, tile layout above
  */
-int svdq_pack_residual(const float* R, int64_t K, int64_t N, uint8_t* r_codes,
-                       uint8_t* r_scales, void* stream);
+svdq_status svdq_pack_residual(const float* R, int64_t K, int64_t N, uint8_t* r_codes,
+                               uint8_t* r_scales, void* stream);
+
+/*
+ * Workspace of svdq_quantize_act for these sizes on the current device, in
+ * bytes (0 when the call needs none: r == 0, or enough rows that no tile is
+ * split along K).  Host-only.
+ */
+svdq_status svdq_quantize_act_workspace(int64_t M, int64_t K, int64_t r, size_t* bytes);
 
 /*
  * Activation step of one forward pass: smoothing, 4-bit quantisation and the
@@ -98,13 +111,21 @@ int svdq_pack_residual(const float* R, int64_t K, int64_t N, uint8_t* r_codes,
  *   x_scales   uint8, svdq_packed_sizes(M, K) output: scales of Xh
  *   T          bf16 [M][r]  output: bf16(bf16(Xh) L1), fp32 accumulation
  *                           (NULL iff r == 0)
+ *   workspace  device scratch of at least svdq_quantize_act_workspace()
+ *              bytes, 16-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE
+ *              (NULL allowed when that size is 0).  When there are fewer
+ *              128-row tiles than SMs, the CTAs sharing a tile sum their
+ *              partial T there in a fixed order; the call leaves the
+ *              workspace's counters at zero again, so one zero fill serves
+ *              all later calls.  Calls that may run concurrently (other
+ *              streams) need workspaces of their own.
  * NVFP4 group rule (16 values v along K): s = E4M3_RNE_satfinite(
  * RN_f32(amax / 6)); rcp = RN_f32(1 / decode(s)) (0 if decode(s) == 0);
  * q_i = E2M1_RNE_satfinite(RN_f32(v_i * rcp)).
  */
-int svdq_quantize_act(const void* X, const float* inv_lambda, const void* L1, int64_t M,
-                      int64_t K, int64_t r, uint8_t* x_codes, uint8_t* x_scales, void* T,
-                      void* stream);
+svdq_status svdq_quantize_act(const void* X, const float* inv_lambda, const void* L1, int64_t M,
+                              int64_t K, int64_t r, uint8_t* x_codes, uint8_t* x_scales, void* T,
+                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Fused 4-bit linear: Y = deq(x) deq(R)^T + T L2 + bias, written as bf16.
@@ -118,10 +139,44 @@ int svdq_quantize_act(const void* X, const float* inv_lambda, const void* L1, in
  *   bias                bf16 [N] or NULL
  *   Y                   bf16 [M][N] output
  */
-int svdq_linear(const uint8_t* x_codes, const uint8_t* x_scales, const void* T,
-                const uint8_t* r_codes, const uint8_t* r_scales, const void* L2,
-                const void* bias, int64_t M, int64_t K, int64_t N, int64_t r, void* Y,
-                void* stream);
+svdq_status svdq_linear(const uint8_t* x_codes, const uint8_t* x_scales, const void* T,
+                        const uint8_t* r_codes, const uint8_t* r_scales, const void* L2,
+                        const void* bias, int64_t M, int64_t K, int64_t N, int64_t r, void* Y,
+                        void* stream);
+
+/*
+ * LoRA adapter joined to the low-rank branch, on the device (chattools.cn
+ * article 584, "main functions", item LoRA integration: adapters apply to
+ * the quantised model without re-quantising it).  With Xh = X
+ * diag(lambda)^-1, the adapter A [K][ra], B [ra][N] (bf16) joins as
+ *     L1_out [K][r + ra] = [L1 | bf16(RN_f32(lambda_k * A_kj))]
+ *     L2_out [r + ra][N] = [L2 ; B]
+ * so that Xh L1_out L2_out = Xh L1 L2 + X A B; the packed residual is
+ * unchanged and the layer then runs with rank r + ra through
+ * svdq_quantize_act / svdq_linear.  Adapters chain: the outputs may be the
+ * inputs of a further call.  Swapping an adapter is a call with the base L1,
+ * L2 and another A, B.
+ *   L1, L2     bf16 [K][r], [r][N] (both NULL iff r == 0)
+ *   lambda     fp32 [K], the smoothing factors (not their reciprocals)
+ *   A, B       bf16 [K][ra], [ra][N]
+ *   L1_out, L2_out  outputs, caller-allocated; must not overlap the inputs
+ * r and ra multiples of 16 with r + ra <= 128, N a multiple of 16.
+ */
+svdq_status svdq_attach_lora(const void* L1, const void* L2, const float* lambda, const void* A,
+                             const void* B, int64_t K, int64_t N, int64_t r, int64_t ra, void* L1_out,
+                             void* L2_out, void* stream);
+
+/*
+ * Kernel choice of svdq_linear (host-side setting for the whole process):
+ *   0  by shape (default): the large-M kernel (persistent CTA pairs, 256 x
+ *      256 tiles over all of K) when its tiles keep at least half of the CTA
+ *      pairs busy, else the small-M kernel (128 x 128 tiles with K split
+ *      over a cluster and summed in distributed shared memory);
+ *   1  always the large-M kernel;   2  always the small-M kernel.
+ * Both compute the same Y (the small-M kernel's fp32 sum runs in another
+ * order).  Returns SVDQ_ERR_INVALID_ARG for any other value.
+ */
+svdq_status svdq_set_linear_path(int path);
 
 /*
  * Failure detection.  Every wait inside the kernels is bounded (default
@@ -134,12 +189,17 @@ int svdq_linear(const uint8_t* x_codes, const uint8_t* x_scales, const void* T,
  * an error) and clears it.  `where`, if not NULL, receives the id of the
  * wait that expired (0 if none).
  */
-int svdq_sync_status(void* stream, int* where);
+svdq_status svdq_sync_status(void* stream, int* where);
+
+/* Sets the limit of every bounded wait in kernels launched from now on, in
+ * nanoseconds (0 < timeout_ns <= 60 s), for all devices of the process.
+ * Host-side setting only; returns SVDQ_ERR_INVALID_ARG outside that range. */
+svdq_status svdq_set_wait_timeout(uint64_t timeout_ns);
 
 /* Self test of the bounded wait: launches one CTA that waits on a barrier
  * nothing will complete, with the given limit in nanoseconds; the wait
  * expires and records SVDQ_ERR_TIMEOUT, read back with svdq_sync_status. */
-int svdq_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
+svdq_status svdq_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
 
 #ifdef __cplusplus
 }

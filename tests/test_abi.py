@@ -76,14 +76,37 @@ def test_linear_validation(lib):
 def test_quantize_and_pack_validation(lib):
     P = ctypes.c_void_p
     q = lib.svdq_quantize_act
-    assert q(P(FAKE), P(FAKE), P(FAKE), 16, 64, 16, P(FAKE), P(FAKE), None, None) == 1  # T missing
-    assert q(P(FAKE), P(FAKE), None, 16, 96, 0, P(FAKE), P(FAKE), None, None) == 2
-    assert q(P(FAKE + 4), P(FAKE), None, 16, 64, 0, P(FAKE), P(FAKE), None, None) == 3
+    assert q(P(FAKE), P(FAKE), P(FAKE), 16, 64, 16, P(FAKE), P(FAKE), None, None, 0, None) == 1  # T missing
+    assert q(P(FAKE), P(FAKE), None, 16, 96, 0, P(FAKE), P(FAKE), None, None, 0, None) == 2
+    assert q(P(FAKE + 4), P(FAKE), None, 16, 64, 0, P(FAKE), P(FAKE), None, None, 0, None) == 3
+    assert q(P(FAKE), P(FAKE), None, 16, 64, 0, P(FAKE), P(FAKE), None, P(FAKE + 8), 64, None) == 3
     p = lib.svdq_pack_residual
     assert p(None, 64, 16, P(FAKE), P(FAKE), None) == 1
     assert p(P(FAKE), 64, 8, P(FAKE), P(FAKE), None) == 2
     assert p(P(FAKE), 64, 16, P(FAKE + 1), P(FAKE), None) == 3
     assert lib.svdq_selftest_wait_timeout(0, None) == 1
+    assert lib.svdq_set_wait_timeout(0) == 1
+    assert lib.svdq_set_wait_timeout(61_000_000_000) == 1
+
+
+def test_size_limits_are_rejected_on_the_host(lib):
+    """M, N <= 2^22 and K <= 2^20 keep every grid dimension and index of the
+    kernels in range; beyond that the calls refuse with UNSUPPORTED_SHAPE."""
+    P = ctypes.c_void_p
+    big_k = (1 << 20) + 64
+    assert lib.svdq_pack_residual(P(FAKE), big_k, 16, P(FAKE), P(FAKE), None) == 2
+    assert lib.svdq_pack_residual(P(FAKE), 64, (1 << 22) + 16, P(FAKE), P(FAKE), None) == 2
+    q = lib.svdq_quantize_act
+    assert q(P(FAKE), P(FAKE), None, (1 << 22) + 1, 64, 0, P(FAKE), P(FAKE), None, None, 0, None) == 2
+    assert q(P(FAKE), P(FAKE), None, 16, big_k, 0, P(FAKE), P(FAKE), None, None, 0, None) == 2
+    lin = lib.svdq_linear
+    args = lambda M, K, N: (P(FAKE), P(FAKE), None, P(FAKE), P(FAKE), None, None, M, K, N, 0, P(FAKE), None)
+    assert lin(*args((1 << 22) + 1, 64, 16)) == 2
+    assert lin(*args(16, big_k, 16)) == 2
+    assert lin(*args(16, 64, (1 << 22) + 16)) == 2
+    from bit_w4a4_quantized_smooth_b200 import packed_sizes, SvdqError
+    with pytest.raises(SvdqError):
+        packed_sizes(16, big_k)
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
@@ -92,3 +115,16 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "_LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         binding.load()
+
+
+def test_attach_lora_validation(lib):
+    P = ctypes.c_void_p
+    f = lib.svdq_attach_lora
+    ok = (P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), 64, 32, 16, 16, P(FAKE), P(FAKE), None)
+    bad = lambda i, v: tuple(v if j == i else a for j, a in enumerate(ok))
+    assert f(*bad(3, None)) == 1        # A missing
+    assert f(*bad(0, None)) == 1        # L1 missing with r > 0
+    assert f(*bad(8, 8)) == 2           # ra not a multiple of 16
+    assert f(*bad(7, 128)) == 2         # r + ra > 128
+    assert f(*bad(6, 24)) == 2          # N not a multiple of 16
+    assert f(*bad(2, P(FAKE + 4))) == 3 # lambda misaligned

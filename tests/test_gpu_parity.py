@@ -120,8 +120,19 @@ def test_quantize_act(case):
     assert svdq.sync_status()[0] == 0
 
 
+@pytest.fixture(params=["large", "small"])
+def linear_path(request):
+    """Each linear test runs through both kernels of svdq_linear: the
+    large-M kernel (CTA pairs, all of K per tile) and the small-M kernel (K
+    split over a cluster, partial sums meeting in distributed shared memory)."""
+    svdq = _lib()
+    svdq.set_linear_path(request.param)
+    yield request.param
+    svdq.set_linear_path("auto")
+
+
 @pytest.mark.parametrize("case", SMALL, ids=_ids)
-def test_linear_on_oracle_operands(case):
+def test_linear_on_oracle_operands(case, linear_path):
     """The GEMM alone: the oracle's packed operands in, Y compared."""
     torch = _torch()
     svdq = _lib()
@@ -144,7 +155,7 @@ def test_linear_on_oracle_operands(case):
 
 
 @pytest.mark.parametrize("case", SMALL, ids=_ids)
-def test_layer_end_to_end(case):
+def test_layer_end_to_end(case, linear_path):
     """quantize_act + linear on the GPU vs the oracle's Y; also the
     quantisation error against the unquantised X W (reported)."""
     torch = _torch()
@@ -162,9 +173,19 @@ def test_layer_end_to_end(case):
     ref = oracle.linear_rows(oxc, oxs, oT, orc, ors, p.L2, p.bias, p.M, p.K, p.N, p.r, rows)
     err = rel_fro(Yg, ref)
     assert err <= Y_TOL, err
-    E = abs_terms(oxc, oxs, oT, orc, ors, p.L2, p.bias, p.M, p.K, p.N, p.r, rows)
-    check_Y_elementwise(Yg, ref, E, p.K, p.r)
+    _check_linear_elementwise(Yg, oxc, oxs, T, orc, ors, p, rows)
     assert svdq.sync_status()[0] == 0
+
+
+def _check_linear_elementwise(Yg_rows, oxc, oxs, T_gpu, orc, ors, p, rows):
+    """The per-element bound of the linear step, given the T the GPU's own
+    activation step produced (T itself is checked against the oracle by
+    check_T, where a rounding flip of one bf16 ulp is allowed; through L2 a
+    flip moves Y by |dT| |L2|, which is T's tolerance, not the linear's)."""
+    Tg = None if T_gpu is None else bf16_to_np_bits(T_gpu)
+    ref = oracle.linear_rows(oxc, oxs, Tg, orc, ors, p.L2, p.bias, p.M, p.K, p.N, p.r, rows)
+    E = abs_terms(oxc, oxs, Tg, orc, ors, p.L2, p.bias, p.M, p.K, p.N, p.r, rows)
+    check_Y_elementwise(Yg_rows, ref, E, p.K, p.r)
 
 
 def test_back_to_back_calls_reuse_outputs():
@@ -237,13 +258,12 @@ def _layer_vs_oracle_rows(p, rows):
     per_row = np.linalg.norm(Yg - ref, axis=1) / np.linalg.norm(ref, axis=1)
     assert per_row.max() <= 2 * Y_TOL, per_row.max()
     # and every sampled element
-    E = abs_terms(oxc, oxs, oT, orc, ors, p.L2, p.bias, p.M, p.K, p.N, p.r, rows)
-    check_Y_elementwise(Yg, ref, E, p.K, p.r)
+    _check_linear_elementwise(Yg, oxc, oxs, T, orc, ors, p, rows)
     return err
 
 
 @pytest.mark.parametrize("case", MULTI, ids=_ids)
-def test_layer_multi_tile(case):
+def test_layer_multi_tile(case, linear_path):
     p = prepare(*case)
     _layer_vs_oracle_rows(p, _sample_rows(p.M))
 

@@ -11,7 +11,7 @@ import pytest
 
 import oracle
 from svdq_inputs import make_layer_inputs
-from svdq_inputs.workloads import make_lora
+from svdq_inputs.workloads import make_lora  # noqa: E402
 from tests._cases import bf16_bits_to_f64, prepare
 
 CASE = ("flux_qkv", 200, 320, 272, 32)
@@ -107,3 +107,28 @@ def test_gpu_layer_with_lora_matches_oracle():
     ref = oracle.linear_rows(oxc, oxs, oT, orc, ors, L2n, p.bias, p.M, p.K, p.N, r2, np.arange(p.M))
     err = rel_fro(bf16_bits_to_f64(bf16_to_np_bits(Y)), ref)
     assert err <= Y_TOL, err
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("r", [0, 32])
+def test_gpu_attach_lora_matches_oracle_bit_exact(r):
+    """svdq_attach_lora (device-side join) equals the oracle's join bit for
+    bit, also with no SVD branch (r = 0) and with a second adapter chained
+    onto the first."""
+    import torch
+    import bit_w4a4_quantized_smooth_b200 as svdq
+    p = prepare(*CASE)
+    L1 = p.L1 if r else None
+    L2 = p.L2 if r else None
+    A, B = _lora(p)
+    A2, B2 = make_lora(0x5EED7001, p.K, p.N, 16)
+    t = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+    bits = lambda x: x.cpu().view(torch.int16).numpy().view(np.uint16)
+    lam = torch.from_numpy(p.lam).cuda()
+    L1g, L2g = svdq.attach_lora(t(L1), t(L2), lam, t(A), t(B))
+    L1h, L2h = svdq.attach_lora(L1g, L2g, lam, t(A2), t(B2))
+    torch.cuda.synchronize()
+    L1n, L2n = oracle.attach_lora(L1, L2, p.lam, A, B)
+    L1m, L2m = oracle.attach_lora(L1n, L2n, p.lam, A2, B2)
+    assert np.array_equal(bits(L1g), L1n) and np.array_equal(bits(L2g), L2n)
+    assert np.array_equal(bits(L1h), L1m) and np.array_equal(bits(L2h), L2m)

@@ -96,3 +96,39 @@ def test_lowrank_rank_zero_is_the_smoothed_weight():
     assert L1 is None and L2 is None
     Wh = (lam.double().numpy()[:, None] * bf16_bits_to_f32(li.W).astype(np.float64)).astype(np.float32)
     assert np.array_equal(R.numpy(), Wh)
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: c[0])
+def test_randomized_lowrank_reconstructs_and_captures_the_top_subspace(case):
+    """The randomized range finder gives a residual that reconstructs Wh to
+    half an fp32 ulp (by construction) and whose spectral norm is within a
+    few percent of sigma_{r+1} (Halko et al., Thm. 10.6: with 2 power
+    iterations and 16 extra samples the excess is a small multiple of
+    sigma_{r+1} for these spectra); missing a planted direction would leave
+    sigma_1-sized residue."""
+    from bit_w4a4_quantized_smooth_b200 import prep
+    name, M, K, N, r = case
+    li = make_layer_inputs(name, M=M, K=K, N=N, r=r)
+    lam, _ = prep.smoothing(_t16(li.Xcal), _t16(li.W))
+    L1, L2, R = prep.lowrank_randomized(_t16(li.W), lam, li.r)
+    assert tuple(L1.shape) == (li.K, li.r) and tuple(L2.shape) == (li.r, li.N)
+    Wh = lam.double().numpy()[:, None] * bf16_bits_to_f32(li.W).astype(np.float64)
+    Rn = R.numpy().astype(np.float64)
+    half_ulp = np.spacing(np.abs(R.numpy())).astype(np.float64) / 2
+    assert np.all(np.abs(_f64(L1) @ _f64(L2) + Rn - Wh) <= half_ulp * (1 + 1e-9) + 1e-300)
+    s = np.linalg.svd(Wh, compute_uv=False)
+    rn = np.linalg.norm(Rn, 2)
+    assert s[li.r] * (1 - 1e-6) <= rn <= 1.1 * s[li.r] + 2.0 ** -7 * s[0], (rn, s[li.r], s[0])
+
+
+def test_randomized_lowrank_is_exact_on_exact_rank():
+    """A weight of rank exactly r is recovered (residual = the bf16
+    rounding of the factors only)."""
+    from bit_w4a4_quantized_smooth_b200 import prep
+    rng = np.random.default_rng(5)
+    K, N, r = 96, 160, 8
+    W = torch.from_numpy(rng.standard_normal((K, r)) @ rng.standard_normal((r, N))).to(torch.bfloat16)
+    lam = torch.ones(K)
+    L1, L2, R = prep.lowrank_randomized(W, lam, r)
+    Wd = W.double().numpy()
+    assert np.linalg.norm(R.numpy().astype(np.float64), 2) <= 2.0 ** -7 * np.linalg.norm(Wd, 2)
