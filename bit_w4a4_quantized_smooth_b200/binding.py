@@ -62,6 +62,8 @@ def load() -> ctypes.CDLL:
         L.svdq_selftest_wait_timeout.argtypes = [ctypes.c_uint64, _P]
         L.svdq_set_wait_timeout.restype = ctypes.c_int
         L.svdq_set_wait_timeout.argtypes = [ctypes.c_uint64]
+        L.svdq_quantize_act_noalloc.restype = ctypes.c_int
+        L.svdq_quantize_act_noalloc.argtypes = [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P]
         L.svdq_attach_lora.restype = ctypes.c_int
         L.svdq_attach_lora.argtypes = [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P]
         L.svdq_set_linear_path.restype = ctypes.c_int
@@ -170,6 +172,25 @@ def linear(x_codes, x_scales, T, r_codes, r_scales, L2, bias, M: int, K: int, N:
                               _ptr(L2), _ptr(bias), M, K, N, r, _ptr(Y), _stream(stream)),
            "svdq_linear")
     return Y
+
+
+def quantize_act_noalloc(X, inv_lambda, L1, x_codes=None, x_scales=None, T=None, stream=None):
+    """quantize_act with its scratch inside the library (svdq_quantize_act_noalloc):
+    for callers that cannot allocate device memory or pass a workspace.  The
+    outputs are allocated here only when not given."""
+    import torch
+    M, K = X.shape
+    r = 0 if L1 is None else L1.shape[1]
+    cb, sb = packed_sizes(M, K)
+    if x_codes is None:
+        x_codes = torch.empty((M, K // 2), dtype=torch.uint8, device=X.device)
+    if x_scales is None:
+        x_scales = torch.empty(sb, dtype=torch.uint8, device=X.device)
+    if T is None and r > 0:
+        T = torch.empty((M, r), dtype=torch.bfloat16, device=X.device)
+    _check(load().svdq_quantize_act_noalloc(_ptr(X), _ptr(inv_lambda), _ptr(L1), M, K, r, _ptr(x_codes),
+                                            _ptr(x_scales), _ptr(T), _stream(stream)), "svdq_quantize_act_noalloc")
+    return x_codes, x_scales, T
 
 
 def attach_lora(L1, L2, lam, A, B, L1_out=None, L2_out=None, stream=None):

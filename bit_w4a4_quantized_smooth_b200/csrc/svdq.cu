@@ -612,4 +612,55 @@ svdq_status svdq_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
   return launch_status();
 }
 
+// ------------------------------------------------ allocation-free variant --
+// svdq_quantize_act with its scratch in a fixed array of this library instead
+// of a caller's buffer, for callers that can neither allocate device memory
+// nor pass scratch (see include/svdq.h).  Every device that loads the library
+// holds the array until the process exits.
+}  // extern "C"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on `dev` (the current device), set up
+// on the first call there: the array's host-side name is only a stand-in, so
+// the address comes from cudaGetSymbolAddress with the device current, and the
+// array is zero-filled once (the counters of the partial-sum exchange must
+// start at zero; every call leaves them at zero again).
+svdq_status noalloc_scratch(int dev, void** ptr) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SVDQ_ERR_CUDA;
+    if (cudaMemset(p, 0, kNoAllocScratchBytes) != cudaSuccess) return SVDQ_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return SVDQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+svdq_status svdq_quantize_act_noalloc(const void* X, const float* inv_lambda, const void* L1, int64_t M, int64_t K,
+                                      int64_t r, uint8_t* x_codes, uint8_t* x_scales, void* T, void* stream) {
+  size_t need = 0;
+  if (svdq_status rc = svdq_quantize_act_workspace(M, K, r, &need)) return rc;
+  if (need > kNoAllocScratchBytes) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  void* scratch = nullptr;
+  if (need > 0) {
+    const int dev = current_device();
+    if (dev < 0) return SVDQ_ERR_CUDA;
+    if (svdq_status rc = noalloc_scratch(dev, &scratch)) return rc;
+  }
+  return svdq_quantize_act(X, inv_lambda, L1, M, K, r, x_codes, x_scales, T, scratch, need ? kNoAllocScratchBytes : 0,
+                           stream);
+}
+
 }  // extern "C"

@@ -201,6 +201,32 @@ svdq_status svdq_set_wait_timeout(uint64_t timeout_ns);
  * expires and records SVDQ_ERR_TIMEOUT, read back with svdq_sync_status. */
 svdq_status svdq_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
 
+/*
+ * svdq_quantize_act without a workspace argument, for callers that can
+ * neither allocate device memory nor hand the library scratch: for example a
+ * plugin inside a host inference engine that owns all device memory and
+ * gives its plugins no scratch, or serving code that may not allocate on its
+ * request path (an allocation can synchronise the device or fail under
+ * memory pressure).  The SVDQuant pages have no counterpart to this call; it
+ * only changes where the activation step keeps its scratch.
+ *
+ * Same arguments and results as svdq_quantize_act, minus the workspace.
+ * The scratch is a fixed 8 MiB array inside the library (every GPU that
+ * loads the library holds it until the process exits), so:
+ *  - shapes whose svdq_quantize_act_workspace() exceeds 8 MiB are refused
+ *    with SVDQ_ERR_UNSUPPORTED_SHAPE (e.g. M = 4608 fits up to r = 64);
+ *  - the first call on a device that needs scratch sets it up (looks up the
+ *    array's device address and zero-fills it, synchronously), so make that
+ *    first call before any stream capture;
+ *  - all calls share the one array, and each leaves its counters at zero for
+ *    the next: calls that may overlap on the GPU (other streams, other host
+ *    threads) race with each other and must be serialised by the caller.
+ * The call allocates no memory (no cudaMalloc, no cudaFree).
+ */
+svdq_status svdq_quantize_act_noalloc(const void* X, const float* inv_lambda, const void* L1,
+                                      int64_t M, int64_t K, int64_t r, uint8_t* x_codes,
+                                      uint8_t* x_scales, void* T, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
