@@ -60,7 +60,7 @@ struct LinParams {
 };
 
 // FULL_K: K is a multiple of 256, every FP4 stage has four K blocks and
-// runs a straight-line issue sequence (scale copies, then four MMAs).
+// runs a straight-line issue sequence.
 template <bool FULL_K>
 __global__ void __launch_bounds__(kLinThreads, 1)
     linear_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_rc,
@@ -237,32 +237,17 @@ __global__ void __launch_bounds__(kLinThreads, 1)
           } else {
             const uint32_t sfa_s = b_s + kLinBBytes;
             const uint32_t sfb_s = sfa_s + kLinSfaBytes;
-            if constexpr (FULL_K) {
-              // copies first, then the MMAs: copies issued back to back cost
-              // the tensor pipe far less than copies interleaved with MMAs
-              const uint32_t first = (it > 0) ? 1u : 0u;
+            // per K block: its three scale copies, then its MMA (measured on
+            // B200: 4% less tensor-pipe time per stage than all twelve copies
+            // ahead of the four MMAs)
+            const int nkb = FULL_K ? 4 : min(4, (K - (it - n_lr) * kLinBK) / 64);
 #pragma unroll
-              for (int kb = 0; kb < 4; ++kb)
-                e_tmem_cp_pair_32x128b_warpx4(sfa_t + 4 * kb, make_sdesc(sfa_s + kb * 512, 0, 128, 0));
-#pragma unroll
-              for (int kb = 0; kb < 4; ++kb) {
-                e_tmem_cp_pair_32x128b_warpx4(sfb_t + 8 * kb, make_sdesc(sfb_s + kb * 512, 0, 128, 0));
-                e_tmem_cp_pair_32x128b_warpx4(sfb_t + 8 * kb + 4, make_sdesc(sfb_s + 2048 + kb * 512, 0, 128, 0));
-              }
-#pragma unroll
-              for (int kb = 0; kb < 4; ++kb)
-                e_mma_nvf4_pair(acc, make_sdesc(a_s + kb * 32, 16, 1024, 2), make_sdesc(b_s + kb * 32, 16, 1024, 2),
-                                idesc_f4, sfa_t + 4 * kb, sfb_t + 8 * kb, kb > 0 ? 1u : first);
-            } else {
-              const int k0 = (it - n_lr) * kLinBK;
-              const int nkb = min(4, (K - k0) / 64);
-              for (int kb = 0; kb < nkb; ++kb) {
-                e_tmem_cp_pair_32x128b_warpx4(sfa_t + 4 * kb, make_sdesc(sfa_s + kb * 512, 0, 128, 0));
-                e_tmem_cp_pair_32x128b_warpx4(sfb_t + 8 * kb, make_sdesc(sfb_s + kb * 512, 0, 128, 0));
-                e_tmem_cp_pair_32x128b_warpx4(sfb_t + 8 * kb + 4, make_sdesc(sfb_s + 2048 + kb * 512, 0, 128, 0));
-                e_mma_nvf4_pair(acc, make_sdesc(a_s + kb * 32, 16, 1024, 2), make_sdesc(b_s + kb * 32, 16, 1024, 2),
-                                idesc_f4, sfa_t + 4 * kb, sfb_t + 8 * kb, (it > 0 || kb > 0) ? 1u : 0u);
-              }
+            for (int kb = 0; kb < nkb; ++kb) {
+              e_tmem_cp_pair_32x128b_warpx4(sfa_t + 4 * kb, make_sdesc(sfa_s + kb * 512, 0, 128, 0));
+              e_tmem_cp_pair_32x128b_warpx4(sfb_t + 8 * kb, make_sdesc(sfb_s + kb * 512, 0, 128, 0));
+              e_tmem_cp_pair_32x128b_warpx4(sfb_t + 8 * kb + 4, make_sdesc(sfb_s + 2048 + kb * 512, 0, 128, 0));
+              e_mma_nvf4_pair(acc, make_sdesc(a_s + kb * 32, 16, 1024, 2), make_sdesc(b_s + kb * 32, 16, 1024, 2),
+                              idesc_f4, sfa_t + 4 * kb, sfb_t + 8 * kb, (it > 0 || kb > 0) ? 1u : 0u);
             }
           }
           e_commit_pair_both(smem_u32(&empty[s]));
@@ -311,7 +296,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
         if (gi == 0 || gi == 3) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(lead(gi == 0 ? ovl_free : &acc_empty[b]));
+          if (lane == 0) mbar_arrive_remote(lead(gi == 0 ? ovl_free : &acc_empty[b]));
         }
         // staging block (alternating per group) must no longer be read by
         // this warp's previous TMA store

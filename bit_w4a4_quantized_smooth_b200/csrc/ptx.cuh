@@ -176,6 +176,16 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
                : "memory");
 }
 
+// Arrive on a (possibly remote) mbarrier with release at CTA scope.  For a
+// hand-off of tensor memory (tcgen05.wait::ld, tcgen05.fence::before_thread_sync,
+// this arrive; the waiter's tcgen05.fence::after_thread_sync) no generic
+// memory has to be published, and the cluster-scope release above waits for
+// every earlier global store of the thread to complete: under a heavily
+// loaded L2 that took about 0.6 us per arrive on B200.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
