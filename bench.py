@@ -53,6 +53,11 @@ def parse_args():
                     help="no timing: three launches of one kernel on the workload (for profilers)")
     ap.add_argument("--sweep", action="store_true",
                     help="the K = N = 3072 sweep over M and rank: one JSON line per point")
+    ap.add_argument("--stack", action="store_true",
+                    help="the synthetic 12B DiT stack (152 linears, rank 32 + LoRA 32): ms per pass, "
+                         "with the oracle's extrapolated time beside it")
+    ap.add_argument("--no-stack", action="store_true",
+                    help="leave the DiT stack pass out of the default single-GPU line")
     return ap.parse_args()
 
 
@@ -489,6 +494,8 @@ def main():
         return run_once(args)
     if args.sweep:
         return run_sweep(args)
+    if args.stack:
+        return run_stack(args)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -505,6 +512,17 @@ def main():
             out["cpu_baseline"] = {"value": round(v, 6), "unit": UNIT, "cores": thr, "kind": "oracle",
                                    "sample": f"{rows} of {L['M']} rows (activation step + linear), "
                                              f"{secs:.1f} s, fp64 OpenMP"}
+        if world == 1 and not args.no_stack:
+            # the whole synthetic DiT stack, one CUDA graph per pass (3 s of
+            # preparation on the device, well under a second of timing)
+            del L
+            torch.cuda.empty_cache()
+            t0 = time.perf_counter()
+            layers = prepare_stack(torch.device("cuda", local_rank))
+            prep_s = time.perf_counter() - t0
+            g_ms, e_ms, launches = time_stack(layers, torch.device("cuda", local_rank))
+            out["stack"] = stack_summary(layers, g_ms, e_ms, launches, prep_s, load_peaks())
+            del layers
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:
@@ -610,6 +628,189 @@ def run_sweep(args):
                 "bound": "tensor" if flops / (fp4_peak * 1e12) > nbytes / (peaks["hbm_gbs"] * 1e9) else "hbm",
                 "roofline_frac": round(roof_us / us, 4), "reps": reps,
                 "l2": "flushed before every rep"}), flush=True)
+    return 0
+
+
+STACK_M = 4608
+
+
+def stack_shape_counts():
+    """{(K, N): number of stack layers of that shape}."""
+    from svdq_inputs import stack_layer_shapes
+    counts = {}
+    for K, N, _ in stack_layer_shapes():
+        counts[(K, N)] = counts.get((K, N), 0) + 1
+    return counts
+
+
+def prepare_stack(device, M=STACK_M, layer_ids=None):
+    """Draw and prepare the layers of the synthetic DiT stack (all 152 by
+    default) on the device, untimed: smoothing on the layer's own
+    activations, rank-32 randomized SVD, the rank-32 LoRA adapter joined to
+    the low-rank branch (effective rank 64, R not re-quantised), R packed to
+    NVFP4."""
+    import torch
+    import bit_w4a4_quantized_smooth_b200 as svdq
+    from bit_w4a4_quantized_smooth_b200 import prep
+    from svdq_inputs import stack_layer_shapes, torch_gen
+    layers = []
+    for i in (range(len(stack_layer_shapes())) if layer_ids is None else layer_ids):
+        d = torch_gen.make_stack_layer(i, M, device)
+        lam, inv = prep.smoothing(d["X"], d["W"])
+        L1, L2, R = prep.lowrank_randomized(d["W"], lam, 32, seed=i)
+        del d["W"]
+        L1, L2 = svdq.attach_lora(L1, L2, lam, d["A"], d["B"])
+        rc, rs = svdq.pack_residual(R)
+        del R
+        layers.append(dict(X=d["X"], inv=inv, L1=L1, L2=L2, rc=rc, rs=rs, K=d["K"], N=d["N"]))
+    torch.cuda.synchronize()
+    return layers
+
+
+def stack_pass_fn(layers, device, M=STACK_M, Y_out=None):
+    """One pass over the stack in layer order on the current stream, into
+    buffers shared by all layers (sized for the widest): the activation
+    codes, scales and T of layer i are consumed by its linear before layer
+    i + 1 overwrites them.  Y goes to one shared buffer too, or to the
+    per-layer tensors of `Y_out`.  Allocates nothing when called."""
+    import torch
+    import bit_w4a4_quantized_smooth_b200 as svdq
+    from bit_w4a4_quantized_smooth_b200 import binding
+    Kmax = max(L["K"] for L in layers)
+    Nmax = max(L["N"] for L in layers)
+    rmax = max(L["L1"].shape[1] for L in layers)
+    xc = torch.empty(M * Kmax // 2, dtype=torch.uint8, device=device)
+    xs = torch.empty(svdq.packed_sizes(M, Kmax)[1], dtype=torch.uint8, device=device)
+    T = torch.empty(M * rmax, dtype=torch.bfloat16, device=device)
+    Y = torch.empty(M * Nmax, dtype=torch.bfloat16, device=device)
+    ws_bytes = max(binding.quantize_act_workspace_bytes(M, L["K"], L["L1"].shape[1]) for L in layers)
+    ws = torch.zeros(max(ws_bytes, 1 << 20), dtype=torch.uint8, device=device)
+    views = []
+    for L in layers:
+        K, N, r = L["K"], L["N"], L["L1"].shape[1]
+        views.append((xc[: M * K // 2].view(M, K // 2), xs[: svdq.packed_sizes(M, K)[1]],
+                      T[: M * r].view(M, r), Y[: M * N].view(M, N) if Y_out is None else Y_out[len(views)]))
+
+    def run():
+        for L, (xck, xsk, Tk, Yk) in zip(layers, views):
+            svdq.quantize_act(L["X"], L["inv"], L["L1"], x_codes=xck, x_scales=xsk, T=Tk, workspace_buf=ws)
+            svdq.linear(xck, xsk, Tk, L["rc"], L["rs"], L["L2"], None, M, L["K"], L["N"], Y=Yk)
+    return run
+
+
+def stack_roofline_ms(layers, peaks, M=STACK_M):
+    """Sum over the layers of each layer's roofline time (the slower of its
+    FP4 FLOPs at the measured FP4 peak and its bytes at the measured HBM
+    rate)."""
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    tot = 0.0
+    for L in layers:
+        K, N, r = L["K"], L["N"], L["L1"].shape[1]
+        tot += max(layer_flops(M, K, N, r) / (fp4_peak * 1e12), linear_bytes(M, K, N, r) / (peaks["hbm_gbs"] * 1e9))
+    return tot * 1e3
+
+
+def time_stack(layers, device, passes=10, warmup=3):
+    """-> (ms per pass replayed from a CUDA graph, ms per pass launched
+    eagerly, launches per pass).  Inputs (10 GB of activations, 3.6 GB of
+    packed weights) are far larger than L2, so no flush is needed."""
+    import torch
+    import bit_w4a4_quantized_smooth_b200 as svdq
+    run = stack_pass_fn(layers, device)
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+
+    def timed(fn, n):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for a, b in ev:
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+    eager_ms = timed(run, max(3, passes // 2))
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(device)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run()  # the capture stream's own warm-up
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        run()
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    graph_ms = timed(g.replay, passes)
+    st, where = svdq.sync_status()
+    if st != 0:
+        raise RuntimeError(f"kernel wait expired in the stack (id {where})")
+    del g
+    return graph_ms, eager_ms, 2 * len(layers)
+
+
+def stack_summary(layers, graph_ms, eager_ms, launches, prep_s, peaks, M=STACK_M):
+    flops = sum(layer_flops(M, L["K"], L["N"], L["L1"].shape[1]) for L in layers)
+    roof = stack_roofline_ms(layers, peaks, M)
+    wbytes = sum(L["rc"].numel() + L["rs"].numel() + 2 * (L["L1"].numel() + L["L2"].numel()) for L in layers)
+    return {
+        "workload": "synthetic 12B DiT stack: 19 double-stream blocks (QKV 3072->9216, out 3072->3072, "
+                    "MLP 3072->12288->3072) + 38 single-stream blocks (fused 3072->21504, 15360->3072), "
+                    f"M={M}, rank 32 + LoRA 32 (effective 64), no bias",
+        "layers": len(layers), "ms_per_pass": round(graph_ms, 3), "ms_per_pass_eager": round(eager_ms, 3),
+        "tflops": round(flops / (graph_ms * 1e-3) / 1e12, 1),
+        "roofline_ms": round(roof, 3), "roofline_frac": round(roof / graph_ms, 4),
+        "gpu_launches_per_pass": launches, "packed_weight_gb": round(wbytes / 1e9, 3),
+        "schedule": "one CUDA graph of the 304 launches (quantize_act + linear per layer), one stream",
+        "prep_s": round(prep_s, 1),
+    }
+
+
+def stack_cpu_baseline(rows=8):
+    """The oracle (activation step + linear, rank 64) timed on `rows` rows of
+    every distinct stack shape, extrapolated by rows and layer counts to the
+    whole pass.  The operands are stand-ins of the right sizes (R = W, zero
+    low-rank factors, unit smoothing): the oracle's cost does not depend on
+    the values.  -> (seconds per pass, threads, sample description)."""
+    import oracle
+    from svdq_inputs import make_stack_layer_inputs, stack_layer_shapes
+    first = {}
+    for i, (K, N, _) in enumerate(stack_layer_shapes()):
+        first.setdefault((K, N), i)
+    r = 64
+    total_s = 0.0
+    for (K, N), n_layers in stack_shape_counts().items():
+        li = make_stack_layer_inputs(first[(K, N)], M=rows)
+        R = (np.asarray(li.W, dtype=np.uint32) << 16).view(np.float32)
+        rc, rs = oracle.pack_residual(R)
+        inv = np.ones(K, dtype=np.float32)
+        L1 = np.zeros((K, r), dtype=np.uint16)
+        L2 = np.zeros((r, N), dtype=np.uint16)
+        t0 = time.perf_counter()
+        xc, xs, T = oracle.quantize_act(li.X[:rows], inv, L1, r)
+        oracle.linear_rows(xc, xs, T, rc, rs, L2, None, rows, K, N, r, np.arange(rows))
+        total_s += (time.perf_counter() - t0) * (STACK_M / rows) * n_layers
+    return total_s, oracle.num_threads(), (f"{rows} rows of each of the {len(first)} distinct layer shapes, "
+                                           f"extrapolated to {STACK_M} rows x 152 layers; stand-in operands")
+
+
+def run_stack(args):
+    import torch
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    t0 = time.perf_counter()
+    layers = prepare_stack(device)
+    prep_s = time.perf_counter() - t0
+    graph_ms, eager_ms, launches = time_stack(layers, device, passes=max(5, min(args.steps, 20)),
+                                              warmup=max(3, args.warmup))
+    out = {"stack": stack_summary(layers, graph_ms, eager_ms, launches, prep_s, load_peaks())}
+    if not args.no_cpu_baseline:
+        secs, thr, sample = stack_cpu_baseline()
+        out["stack"]["cpu_baseline"] = {"ms_per_pass": round(secs * 1e3, 1), "cores": thr, "kind": "oracle",
+                                        "sample": sample}
+    print(json.dumps(out), flush=True)
     return 0
 
 

@@ -104,3 +104,11 @@ def test_step_stats():
     st = bench.step_stats([0.1 + 0.001 * i for i in range(50)])   # 100 .. 149 µs
     assert st["median_us"] == pytest.approx(124.5)
     assert 100.0 <= st["p10_us"] < st["median_us"] < st["p90_us"] <= 149.0
+
+
+def test_stack_shape_counts():
+    import bench
+    counts = bench.stack_shape_counts()
+    assert sum(counts.values()) == 152
+    assert counts == {(3072, 9216): 19, (3072, 3072): 19, (3072, 12288): 19, (12288, 3072): 19,
+                      (3072, 21504): 38, (15360, 3072): 38}
