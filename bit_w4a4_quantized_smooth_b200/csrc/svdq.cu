@@ -509,12 +509,14 @@ svdq_status svdq_linear(const uint8_t* x_codes, const uint8_t* x_scales, const v
     if (rc) return rc;
   }
 
-  // Few rows: the large-M kernel's 256 x 256 pair tiles would keep fewer
-  // than half of the CTA pairs busy, each walking all of K; the small-M
-  // kernel splits K over a cluster instead.
+  // At most 128 rows with tiles for under a quarter of the SMs: the large-M
+  // kernel would leave most SMs idle, each busy pair walking all of K; the
+  // small-M kernel splits K over a cluster instead.  Measured on B200
+  // (K, N in {3072, 12288}): the small-M kernel is faster only there; from
+  // 256 rows, or with N = 12288 at any M, the large-M kernel is.
   const int64_t pair_tiles = ((M + svdq::kLinBM - 1) / svdq::kLinBM) * ((N + svdq::kLinBN - 1) / svdq::kLinBN);
   const int path = g_linear_path.load(std::memory_order_relaxed);
-  if (path == 2 || (path == 0 && pair_tiles < sms / 2))
+  if (path == 2 || (path == 0 && M <= 128 && 4 * pair_tiles < sms))
     return launch_linear_splitk(tm_xc, tm_rc, tm_xs, tm_rs, tm_t, tm_l2, bias, Y, M, K, N, r, dev, sms, stream);
 
   svdq::LinParams p;

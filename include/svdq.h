@@ -168,10 +168,11 @@ svdq_status svdq_attach_lora(const void* L1, const void* L2, const float* lambda
 
 /*
  * Kernel choice of svdq_linear (host-side setting for the whole process):
- *   0  by shape (default): the large-M kernel (persistent CTA pairs, 256 x
- *      256 tiles over all of K) when its tiles keep at least half of the CTA
- *      pairs busy, else the small-M kernel (128 x 128 tiles with K split
- *      over a cluster and summed in distributed shared memory);
+ *   0  by shape (default): the small-M kernel (128 x 128 tiles with K split
+ *      over a cluster and summed in distributed shared memory) for M <= 128
+ *      when the large-M kernel's 256 x 256 tiles would cover fewer than a
+ *      quarter of the SMs, else the large-M kernel (persistent CTA pairs,
+ *      256 x 256 tiles over all of K);
  *   1  always the large-M kernel;   2  always the small-M kernel.
  * Both compute the same Y (the small-M kernel's fp32 sum runs in another
  * order).  Returns SVDQ_ERR_INVALID_ARG for any other value.
