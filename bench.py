@@ -51,6 +51,8 @@ def parse_args():
                     help="target CPU time of the oracle sample")
     ap.add_argument("--once", choices=["quantize_act", "linear", "pack_residual"],
                     help="no timing: three launches of one kernel on the workload (for profilers)")
+    ap.add_argument("--rows", type=int, default=None,
+                    help="with --once: M rows instead of the workload's (same distributions)")
     ap.add_argument("--sweep", action="store_true",
                     help="the K = N = 3072 sweep over M and rank: one JSON line per point")
     ap.add_argument("--stack", action="store_true",
@@ -65,7 +67,7 @@ def parse_args():
 # `bench.py --once linear --workload <name>` (L2-warm), per workload.  A figure
 # is reported only while the kernel sources hash to the captured ones.
 LINEAR_TRAFFIC_CAPTURES = {
-    "flux_qkv": {"bytes": 24844032 + 30347008, "sources_sha256": "f995a861848ff4cb"},
+    "flux_mlp_up": {"bytes": 30408960 + 58434304, "sources_sha256": "36fbc53256e6394a"},
 }
 
 
@@ -172,13 +174,13 @@ def workload_desc(name, M, K, N, r):
             "M": M, "K": K, "N": N, "rank": r, "l2": "flushed before every step (512 MB write, then 256 MB read: cold, clean L2)"}
 
 
-def setup_layer(name: str, device):
+def setup_layer(name: str, device, M=None):
     import torch
     import bit_w4a4_quantized_smooth_b200 as svdq
     from bit_w4a4_quantized_smooth_b200 import prep
     from svdq_inputs import make_layer_inputs
 
-    li = make_layer_inputs(name)
+    li = make_layer_inputs(name, M=M)
 
     def bf16(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
@@ -538,7 +540,7 @@ def run_once(args):
     import bit_w4a4_quantized_smooth_b200 as svdq
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
-    L = setup_layer(args.workload, device)
+    L = setup_layer(args.workload, device, M=args.rows)
     M, K, N, r = L["M"], L["K"], L["N"], L["r"]
     xc, xs, T = svdq.quantize_act(L["X"], L["inv"], L["L1"])
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
