@@ -11,6 +11,7 @@ binding raises if the library is missing.
 from .binding import (  # noqa: F401
     SvdqError,
     attach_lora,
+    channel_absmax,
     lib_path,
     linear,
     load,

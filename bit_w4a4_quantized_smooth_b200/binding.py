@@ -68,6 +68,8 @@ def load() -> ctypes.CDLL:
         L.svdq_attach_lora.argtypes = [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P]
         L.svdq_set_linear_path.restype = ctypes.c_int
         L.svdq_set_linear_path.argtypes = [ctypes.c_int]
+        L.svdq_channel_absmax.restype = ctypes.c_int
+        L.svdq_channel_absmax.argtypes = [_P, _I64, _I64, _P, _P]
         _lib = L
     return _lib
 
@@ -208,6 +210,18 @@ def attach_lora(L1, L2, lam, A, B, L1_out=None, L2_out=None, stream=None):
     _check(load().svdq_attach_lora(_ptr(L1), _ptr(L2), _ptr(lam), _ptr(A), _ptr(B), K, N, r, ra, _ptr(L1_out),
                                    _ptr(L2_out), _stream(stream)), "svdq_attach_lora")
     return L1_out, L2_out
+
+
+def channel_absmax(X, amax=None, stream=None):
+    """Fold a bf16 [M][K] activation batch into the running per-channel
+    max |X| (fp32 [K] on the device; zeros are allocated when `amax` is
+    None).  Returns amax."""
+    import torch
+    M, K = X.shape
+    if amax is None:
+        amax = torch.zeros(K, dtype=torch.float32, device=X.device)
+    _check(load().svdq_channel_absmax(_ptr(X), M, K, _ptr(amax), _stream(stream)), "svdq_channel_absmax")
+    return amax
 
 
 def sync_status(stream=None) -> Tuple[int, int]:

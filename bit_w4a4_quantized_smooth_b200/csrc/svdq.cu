@@ -13,6 +13,7 @@
 #include <unordered_map>
 
 #include "../../include/svdq.h"
+#include "calib.cuh"
 #include "linear.cuh"
 #include "linear_splitk.cuh"
 #include "lora.cuh"
@@ -575,6 +576,28 @@ svdq_status svdq_attach_lora(const void* L1, const void* L2, const float* lambda
       static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B), static_cast<int>(K),
       static_cast<int>(N), static_cast<int>(r), static_cast<int>(ra), static_cast<__nv_bfloat16*>(L1_out),
       static_cast<__nv_bfloat16*>(L2_out));
+  return launch_status();
+}
+
+svdq_status svdq_channel_absmax(const void* X, int64_t M, int64_t K, float* amax, void* stream) {
+  if (!X || !amax || M <= 0 || K <= 0) return SVDQ_ERR_INVALID_ARG;
+  if (K % 8 != 0 || K > kMaxK || M > kMaxRows) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || !aligned16(amax)) return SVDQ_ERR_MISALIGNED;
+  const int dev = current_device();
+  if (dev < 0) return SVDQ_ERR_CUDA;
+  const int sms = sm_count(dev);
+  if (sms <= 0) return SVDQ_ERR_CUDA;
+  // enough row ranges for about four blocks per SM, at least 32 rows each
+  const int64_t col_blocks = (K / 8 + svdq::kAbsmaxThreads - 1) / svdq::kAbsmaxThreads;
+  int64_t row_blocks = (4 * static_cast<int64_t>(sms) + col_blocks - 1) / col_blocks;
+  if (row_blocks > (M + 31) / 32) row_blocks = (M + 31) / 32;
+  if (row_blocks > 65535) row_blocks = 65535;
+  const int64_t rows_per_block = (M + row_blocks - 1) / row_blocks;
+  row_blocks = (M + rows_per_block - 1) / rows_per_block;
+  const dim3 grid(static_cast<unsigned>(col_blocks), static_cast<unsigned>(row_blocks));
+  svdq::channel_absmax_kernel<<<grid, svdq::kAbsmaxThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(X), static_cast<int>(M), static_cast<int>(K),
+      static_cast<int>(rows_per_block), reinterpret_cast<unsigned int*>(amax));
   return launch_status();
 }
 

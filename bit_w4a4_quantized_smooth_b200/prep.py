@@ -22,7 +22,15 @@ import torch
 
 def smoothing(Xcal: torch.Tensor, W: torch.Tensor):
     """-> (lambda fp32 [K], inv_lambda fp32 [K])."""
-    a = Xcal.abs().amax(dim=0).double()
+    return smoothing_from_stats(Xcal.abs().amax(dim=0).float(), W)
+
+
+def smoothing_from_stats(x_amax: torch.Tensor, W: torch.Tensor):
+    """The smoothing factors from calibration statistics: x_amax fp32 [K],
+    the per-channel max |X| over every calibration batch (gathered on the
+    device by svdq_channel_absmax, batch by batch).
+    -> (lambda fp32 [K], inv_lambda fp32 [K])."""
+    a = x_amax.double()
     b = W.abs().amax(dim=1).double()
     lam = torch.where((a == 0) | (b == 0), torch.ones_like(a), a.sqrt() / b.sqrt()).float()
     inv = torch.ones_like(lam) / lam  # fp32 quotient, rounded once

@@ -167,6 +167,23 @@ svdq_status svdq_attach_lora(const void* L1, const void* L2, const float* lambda
                              void* L2_out, void* stream);
 
 /*
+ * Smoothing statistics (chattools.cn article 584, "technical principles":
+ * lambda_k = sqrt(max_i |X_ik|) / sqrt(max_n |W_kn|) takes the largest
+ * magnitude of each input channel over the calibration activations).
+ * Folds one batch into a running per-channel maximum on the device:
+ *     amax[k] = max(amax[k], max_i |X[i][k]|),   i < M.
+ *   X     bf16 [M][K] row-major, device, 16-byte aligned; not modified
+ *   amax  fp32 [K], device, 16-byte aligned, caller-owned; set it to zeros
+ *         before the first batch and pass it unchanged to later ones
+ * The result is exact (a maximum of bf16 magnitudes) and does not depend on
+ * the order of rows or batches; a NaN in X makes its channel's value NaN.
+ * Calls on one amax must be stream-ordered.  K a multiple of 8.
+ * Errors: SVDQ_ERR_INVALID_ARG (null pointer, M or K <= 0),
+ * SVDQ_ERR_UNSUPPORTED_SHAPE, SVDQ_ERR_MISALIGNED, SVDQ_ERR_CUDA.
+ */
+svdq_status svdq_channel_absmax(const void* X, int64_t M, int64_t K, float* amax, void* stream);
+
+/*
  * Kernel choice of svdq_linear (host-side setting for the whole process):
  *   0  by shape (default): the small-M kernel (128 x 128 tiles with K split
  *      over a cluster and summed in distributed shared memory) for M <= 128

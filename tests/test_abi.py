@@ -128,3 +128,13 @@ def test_attach_lora_validation(lib):
     assert f(*bad(7, 128)) == 2         # r + ra > 128
     assert f(*bad(6, 24)) == 2          # N not a multiple of 16
     assert f(*bad(2, P(FAKE + 4))) == 3 # lambda misaligned
+
+
+def test_channel_absmax_validation(lib):
+    P = ctypes.c_void_p
+    f = lib.svdq_channel_absmax
+    assert f(None, 4, 64, P(FAKE), None) == 1            # null X
+    assert f(P(FAKE), 0, 64, P(FAKE), None) == 1         # no rows
+    assert f(P(FAKE), 4, 60, P(FAKE), None) == 2         # K not a multiple of 8
+    assert f(P(FAKE + 4), 4, 64, P(FAKE), None) == 3     # misaligned X
+    assert f(P(FAKE), 4, 64, P(FAKE + 8), None) == 3     # misaligned amax
