@@ -82,6 +82,12 @@ def lib() -> ctypes.CDLL:
             ("oracle_quantize_act", [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P]),
             ("oracle_dequant", [_P, _P, _I64, _I64, _P]),
             ("oracle_linear_rows", [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _I64, _P]),
+            ("oracle_quantize_group_gs", [_P, ctypes.c_float, _P, _P]),
+            ("oracle_quantize_rows_gs", [_P, _I64, _I64, ctypes.c_float, _P, _P]),
+            ("oracle_pack_residual_gs", [_P, _I64, _I64, ctypes.c_float, _P, _P]),
+            ("oracle_quantize_act_gs", [_P, _P, _P, _I64, _I64, _I64, ctypes.c_float, _P, _P, _P]),
+            ("oracle_linear_rows_gs", [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_double,
+                                       ctypes.c_double, _P, _I64, _P]),
         ]:
             f = getattr(L, name)
             f.restype = ctypes.c_int
@@ -135,6 +141,16 @@ def quantize_group(v) -> tuple[np.ndarray, int]:
     return codes, int(s[0])
 
 
+def quantize_group_gs(v, g: float) -> tuple[np.ndarray, int]:
+    """One group of 16 with the two-level quantiser (global scale g > 0)."""
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    assert v.shape == (16,)
+    codes = np.zeros(16, dtype=np.uint8)
+    s = np.zeros(1, dtype=np.uint8)
+    _check(lib().oracle_quantize_group_gs(_ptr(v), float(g), _ptr(codes), _ptr(s)), "quantize_group_gs")
+    return codes, int(s[0])
+
+
 def scale_offset(row: int, g: int, K: int) -> int:
     return lib().oracle_scale_offset(row, g, K)
 
@@ -156,6 +172,28 @@ def quantize_rows(V: np.ndarray):
     codes = np.zeros((rows, K // 2), dtype=np.uint8)
     scales = np.zeros(scale_bytes(rows, K), dtype=np.uint8)
     _check(lib().oracle_quantize_rows(_ptr(V), rows, K, _ptr(codes), _ptr(scales)), "quantize_rows")
+    return codes, scales
+
+
+def quantize_rows_gs(V: np.ndarray, g: float):
+    """fp32 [rows][K] with global scale g -> (codes, scales)."""
+    V = np.ascontiguousarray(V, dtype=np.float32)
+    rows, K = V.shape
+    codes = np.zeros((rows, K // 2), dtype=np.uint8)
+    scales = np.zeros(scale_bytes(rows, K), dtype=np.uint8)
+    _check(lib().oracle_quantize_rows_gs(_ptr(V), rows, K, float(g), _ptr(codes), _ptr(scales)),
+           "quantize_rows_gs")
+    return codes, scales
+
+
+def pack_residual_gs(R: np.ndarray, gw: float):
+    """R fp32 [K][N] with global scale g_w -> (r_codes [N][K/2], r_scales)."""
+    R = np.ascontiguousarray(R, dtype=np.float32)
+    K, N = R.shape
+    codes = np.zeros((N, K // 2), dtype=np.uint8)
+    scales = np.zeros(scale_bytes(N, K), dtype=np.uint8)
+    _check(lib().oracle_pack_residual_gs(_ptr(R), K, N, float(gw), _ptr(codes), _ptr(scales)),
+           "pack_residual_gs")
     return codes, scales
 
 
@@ -247,6 +285,31 @@ def quantize_act(X: np.ndarray, inv_lambda: np.ndarray, L1: Optional[np.ndarray]
     _check(lib().oracle_quantize_act(_ptr(X), _ptr(inv_lambda), _ptr(L1c), M, K, r, _ptr(codes),
                                      _ptr(scales), _ptr(T)), "quantize_act")
     return codes, scales, T
+
+
+def quantize_act_gs(X: np.ndarray, inv_lambda: np.ndarray, L1: Optional[np.ndarray], r: int, gx: float):
+    """The activation step with global scale g_x for Xh (T is of Xh itself)."""
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    inv_lambda = np.ascontiguousarray(inv_lambda, dtype=np.float32)
+    M, K = X.shape
+    codes = np.zeros((M, K // 2), dtype=np.uint8)
+    scales = np.zeros(scale_bytes(M, K), dtype=np.uint8)
+    T = np.zeros((M, r), dtype=np.uint16) if r > 0 else None
+    L1c = None if r == 0 else np.ascontiguousarray(L1, dtype=np.uint16)
+    _check(lib().oracle_quantize_act_gs(_ptr(X), _ptr(inv_lambda), _ptr(L1c), M, K, r, float(gx), _ptr(codes),
+                                        _ptr(scales), _ptr(T)), "quantize_act_gs")
+    return codes, scales, T
+
+
+def linear_rows_gs(x_codes, x_scales, T, r_codes, r_scales, L2, bias, M, K, N, r, gx, gw, rows) -> np.ndarray:
+    """fp64 output rows with global scales: g_x g_w sum deq deq + T L2 + bias."""
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    Y = np.zeros((len(rows), N), dtype=np.float64)
+    args = [np.ascontiguousarray(a) if a is not None else None
+            for a in (x_codes, x_scales, T, r_codes, r_scales, L2, bias)]
+    _check(lib().oracle_linear_rows_gs(*[_ptr(a) for a in args], M, K, N, r, float(gx), float(gw), _ptr(rows),
+                                       len(rows), _ptr(Y)), "linear_rows_gs")
+    return Y
 
 
 def dequant(codes: np.ndarray, scales: np.ndarray, rows: int, K: int) -> np.ndarray:

@@ -144,6 +144,29 @@ void quantize_group(const float* v, int64_t stride, uint8_t* codes, uint8_t* sca
   *scale = s;
 }
 
+// ---------------------------------- NVFP4 with a per-tensor global scale ----
+// Two-level scaling: the tensor carries one fp32 scale g > 0 on top of the
+// per-16 E4M3 scales, and an element dequantises to q * decode(s) * g.  One
+// group of 16 values v (fp32):
+//   amax = max |v_i|
+//   s_f  = RN_f32(amax / 6)
+//   s    = E4M3_RNE_satfinite(RN_f32(s_f * RN_f32(1 / g)))
+//   d    = RN_f32(decode(s) * g)                 (the group's whole scale)
+//   rcp  = 0 if d == 0 else RN_f32(1 / d)
+//   q_i  = E2M1_RNE_satfinite(RN_f32(v_i * rcp))
+// With g = 1 this is quantize_group above.
+void quantize_group_gs(const float* v, int64_t stride, float g, uint8_t* codes, uint8_t* scale) {
+  float amax = 0.0f;
+  for (int i = 0; i < 16; ++i) amax = std::max(amax, std::fabs(v[i * stride]));
+  const float sf = amax / 6.0f;
+  const float inv_g = 1.0f / g;
+  const uint8_t s = e4m3_encode(sf * inv_g);
+  const float d = static_cast<float>(e4m3_decode(s)) * g;
+  const float rcp = (d == 0.0f) ? 0.0f : 1.0f / d;
+  for (int i = 0; i < 16; ++i) codes[i] = e2m1_encode(v[i * stride] * rcp);
+  *scale = s;
+}
+
 // ------------------------------------------------------------- layouts ----
 // Codes: row-major [rows][K/2]; element k of a row sits in byte k/2, in the
 // low nibble when k is even and in the high nibble when k is odd.
@@ -164,16 +187,20 @@ uint8_t code_at(const uint8_t* codes, int64_t row, int64_t k, int64_t K) {
 }
 
 // Quantise `rows` vectors of length K, element (i, k) at V[i*row_stride + k*k_stride],
-// into packed codes and tiled scales.
+// into packed codes and tiled scales; `gs` > 0 selects the two-level
+// quantiser with that global scale, 0 the plain one.
 void quantize_rows(const float* V, int64_t rows, int64_t K, int64_t row_stride, int64_t k_stride,
-                   uint8_t* codes, uint8_t* scales) {
+                   uint8_t* codes, uint8_t* scales, float gs = 0.0f) {
   std::memset(scales, 0, static_cast<size_t>(scale_bytes(rows, K)));
 #pragma omp parallel for schedule(static)
   for (int64_t i = 0; i < rows; ++i) {
     uint8_t q[16];
     for (int64_t g = 0; g < K / 16; ++g) {
       uint8_t s;
-      quantize_group(V + i * row_stride + g * 16 * k_stride, k_stride, q, &s);
+      if (gs > 0.0f)
+        quantize_group_gs(V + i * row_stride + g * 16 * k_stride, k_stride, gs, q, &s);
+      else
+        quantize_group(V + i * row_stride + g * 16 * k_stride, k_stride, q, &s);
       scales[scale_offset(i, g, K)] = s;
       for (int j = 0; j < 16; j += 2)
         codes[i * (K / 2) + g * 8 + j / 2] = static_cast<uint8_t>(q[j] | (q[j + 1] << 4));
@@ -413,11 +440,31 @@ int oracle_quantize_rows(const float* V, int64_t rows, int64_t K, uint8_t* codes
   return 0;
 }
 
+// One group of 16 with the two-level quantiser (global scale g > 0).
+int oracle_quantize_group_gs(const float* v, float g, uint8_t* codes, uint8_t* scale) {
+  if (!(g > 0.0f)) return 1;
+  quantize_group_gs(v, 1, g, codes, scale);
+  return 0;
+}
+
+int oracle_quantize_rows_gs(const float* V, int64_t rows, int64_t K, float g, uint8_t* codes, uint8_t* scales) {
+  if (K % 64 != 0 || rows < 0 || !(g > 0.0f)) return 1;
+  quantize_rows(V, rows, K, K, 1, codes, scales, g);
+  return 0;
+}
+
 // Residual packer (step "pack R"): R fp32 [K][N] row-major; group of 16 along
 // K for every output column n -> r_codes [N][K/2], r_scales tiled (N rows).
 int oracle_pack_residual(const float* R, int64_t K, int64_t N, uint8_t* r_codes, uint8_t* r_scales) {
   if (K % 64 != 0 || N <= 0) return 1;
   quantize_rows(R, N, K, 1, N, r_codes, r_scales);
+  return 0;
+}
+
+// The same with a global scale g_w > 0 for R (two-level NVFP4).
+int oracle_pack_residual_gs(const float* R, int64_t K, int64_t N, float gw, uint8_t* r_codes, uint8_t* r_scales) {
+  if (K % 64 != 0 || N <= 0 || !(gw > 0.0f)) return 1;
+  quantize_rows(R, N, K, 1, N, r_codes, r_scales, gw);
   return 0;
 }
 
@@ -591,14 +638,24 @@ int oracle_attach_lora(const uint16_t* L1, const uint16_t* L2, const float* lamb
 //   Xh  = RN_f32(X * inv_lambda)             per element
 //   (x_codes, x_scales) = NVFP4(Xh) by groups of 16 along K
 //   T   = bf16(sum_k bf16(Xh)_k L1[k][:])    fp64 sum, one rounding
+int oracle_quantize_act_gs(const uint16_t* X, const float* inv_lambda, const uint16_t* L1, int64_t M,
+                           int64_t K, int64_t r, float gx, uint8_t* x_codes, uint8_t* x_scales, uint16_t* T);
+
 int oracle_quantize_act(const uint16_t* X, const float* inv_lambda, const uint16_t* L1, int64_t M,
                         int64_t K, int64_t r, uint8_t* x_codes, uint8_t* x_scales, uint16_t* T) {
-  if (K % 64 != 0 || M < 0) return 1;
+  return oracle_quantize_act_gs(X, inv_lambda, L1, M, K, r, 0.0f, x_codes, x_scales, T);
+}
+
+// The activation step with a global scale g_x for Xh (g_x = 0: the plain
+// quantiser); T is of Xh itself, unaffected by the global scale.
+int oracle_quantize_act_gs(const uint16_t* X, const float* inv_lambda, const uint16_t* L1, int64_t M,
+                           int64_t K, int64_t r, float gx, uint8_t* x_codes, uint8_t* x_scales, uint16_t* T) {
+  if (K % 64 != 0 || M < 0 || gx < 0.0f) return 1;
   std::vector<float> Xh(static_cast<size_t>(M) * K);
 #pragma omp parallel for schedule(static)
   for (int64_t i = 0; i < M; ++i)
     for (int64_t k = 0; k < K; ++k) Xh[i * K + k] = bf16_to_f32(X[i * K + k]) * inv_lambda[k];
-  quantize_rows(Xh.data(), M, K, K, 1, x_codes, x_scales);
+  quantize_rows(Xh.data(), M, K, K, 1, x_codes, x_scales, gx);
   if (r > 0) {
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < M; ++i) {
@@ -626,11 +683,26 @@ int oracle_dequant(const uint8_t* codes, const uint8_t* scales, int64_t rows, in
 // Output rows of the linear layer, in fp64:
 //   Y[m][n] = sum_k deq(x)[m][k] deq(R)[n][k] + sum_j T[m][j] L2[j][n] + bias[n]
 // for the listed rows only (rows[i] in [0, M)).  bias may be NULL.
+int oracle_linear_rows_gs(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* T,
+                          const uint8_t* r_codes, const uint8_t* r_scales, const uint16_t* L2,
+                          const uint16_t* bias, int64_t M, int64_t K, int64_t N, int64_t r, double gx,
+                          double gw, const int64_t* rows, int64_t nrows, double* Y);
+
 int oracle_linear_rows(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* T,
                        const uint8_t* r_codes, const uint8_t* r_scales, const uint16_t* L2,
                        const uint16_t* bias, int64_t M, int64_t K, int64_t N, int64_t r,
                        const int64_t* rows, int64_t nrows, double* Y) {
-  if (K % 64 != 0) return 1;
+  return oracle_linear_rows_gs(x_codes, x_scales, T, r_codes, r_scales, L2, bias, M, K, N, r, 1.0, 1.0, rows,
+                               nrows, Y);
+}
+
+// With global scales: deq(x) and deq(R) carry their tensors' global scales,
+//   Y[m][n] = g_x g_w sum_k q_x s_x q_R s_R + sum_j T[m][j] L2[j][n] + bias[n].
+int oracle_linear_rows_gs(const uint8_t* x_codes, const uint8_t* x_scales, const uint16_t* T,
+                          const uint8_t* r_codes, const uint8_t* r_scales, const uint16_t* L2,
+                          const uint16_t* bias, int64_t M, int64_t K, int64_t N, int64_t r, double gx,
+                          double gw, const int64_t* rows, int64_t nrows, double* Y) {
+  if (K % 64 != 0 || !(gx > 0.0) || !(gw > 0.0)) return 1;
   std::vector<float> Rd(static_cast<size_t>(N) * K);
   oracle_dequant(r_codes, r_scales, N, K, Rd.data());
   for (int64_t t = 0; t < nrows; ++t) {
@@ -646,7 +718,7 @@ int oracle_linear_rows(const uint8_t* x_codes, const uint8_t* x_scales, const ui
       for (int64_t k = 0; k < K; ++k) acc += xd[k] * (double)rd[k];
       double lr = 0.0;
       for (int64_t j = 0; j < r; ++j) lr += (double)bf16_to_f32(T[m * r + j]) * (double)bf16_to_f32(L2[j * N + n]);
-      Y[t * N + n] = acc + lr + (bias ? (double)bf16_to_f32(bias[n]) : 0.0);
+      Y[t * N + n] = gx * gw * acc + lr + (bias ? (double)bf16_to_f32(bias[n]) : 0.0);
     }
   }
   return 0;
