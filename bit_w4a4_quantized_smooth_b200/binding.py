@@ -68,6 +68,9 @@ def load() -> ctypes.CDLL:
         L.svdq_attach_lora.argtypes = [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P]
         L.svdq_set_linear_path.restype = ctypes.c_int
         L.svdq_set_linear_path.argtypes = [ctypes.c_int]
+        L.svdq_linear_scaled.restype = ctypes.c_int
+        L.svdq_linear_scaled.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_float,
+                                         _P, _P]
         L.svdq_channel_absmax.restype = ctypes.c_int
         L.svdq_channel_absmax.argtypes = [_P, _I64, _I64, _P, _P]
         _lib = L
@@ -164,15 +167,21 @@ def quantize_act(X, inv_lambda, L1, x_codes=None, x_scales=None, T=None, stream=
 
 
 def linear(x_codes, x_scales, T, r_codes, r_scales, L2, bias, M: int, K: int, N: int,
-           Y=None, stream=None):
-    """Fused 4-bit linear -> Y bf16 [M][N]."""
+           Y=None, stream=None, alpha: float = 1.0):
+    """Fused 4-bit linear -> Y bf16 [M][N]; `alpha` (a power of two) scales
+    the accumulator before the bias (per-tensor global scales g_x g_w)."""
     import torch
     r = 0 if L2 is None else L2.shape[0]
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.bfloat16, device=x_codes.device)
-    _check(load().svdq_linear(_ptr(x_codes), _ptr(x_scales), _ptr(T), _ptr(r_codes), _ptr(r_scales),
-                              _ptr(L2), _ptr(bias), M, K, N, r, _ptr(Y), _stream(stream)),
-           "svdq_linear")
+    if alpha == 1.0:
+        _check(load().svdq_linear(_ptr(x_codes), _ptr(x_scales), _ptr(T), _ptr(r_codes), _ptr(r_scales),
+                                  _ptr(L2), _ptr(bias), M, K, N, r, _ptr(Y), _stream(stream)),
+               "svdq_linear")
+    else:
+        _check(load().svdq_linear_scaled(_ptr(x_codes), _ptr(x_scales), _ptr(T), _ptr(r_codes), _ptr(r_scales),
+                                         _ptr(L2), _ptr(bias), M, K, N, r, float(alpha), _ptr(Y),
+                                         _stream(stream)), "svdq_linear_scaled")
     return Y
 
 

@@ -54,6 +54,7 @@ constexpr int kLinNumBars = 2 * kLinStages + 2 + 2 + 1 + 1 + 1;
 struct LinParams {
   const __nv_bfloat16* bias;
   __nv_bfloat16* Y;
+  float alpha;  // a power of two: the 4-bit product's global scales g_x g_w (1 without them)
   int M, K, N, r;
   int m_tiles, tiles;  // pair tiles: ceil(M / 256) x ceil(N / 256)
   uint64_t timeout_ns;
@@ -266,6 +267,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     const int q = warp & 3;    // TMEM lane quadrant this warp may access
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     uint8_t* out_s = smem + kLinStageOut + (warp - 2) * 2 * kLinOutBytes;
+    const float alpha = p.alpha;
     int i = 0;
     for (int t = pair; t < p.tiles; t += pairs, ++i) {
       const int b = i & 1;
@@ -307,14 +309,10 @@ __global__ void __launch_bounds__(kLinThreads, 1)
         const float* bs = bias_s + 32 * c0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {  // 16-byte chunk j = columns 8 j .. 8 j + 7
-          const uint4 w = make_uint4(pack_bf16x2(__uint_as_float(v[8 * j + 0]) + bs[8 * j + 0],
-                                                 __uint_as_float(v[8 * j + 1]) + bs[8 * j + 1]),
-                                     pack_bf16x2(__uint_as_float(v[8 * j + 2]) + bs[8 * j + 2],
-                                                 __uint_as_float(v[8 * j + 3]) + bs[8 * j + 3]),
-                                     pack_bf16x2(__uint_as_float(v[8 * j + 4]) + bs[8 * j + 4],
-                                                 __uint_as_float(v[8 * j + 5]) + bs[8 * j + 5]),
-                                     pack_bf16x2(__uint_as_float(v[8 * j + 6]) + bs[8 * j + 6],
-                                                 __uint_as_float(v[8 * j + 7]) + bs[8 * j + 7]));
+          // alpha is a power of two, so the product is exact: Y = bf16(acc alpha + bias)
+          auto y = [&](int e) { return __fmul_rn(__uint_as_float(v[8 * j + e]), alpha) + bs[8 * j + e]; };
+          const uint4 w = make_uint4(pack_bf16x2(y(0), y(1)), pack_bf16x2(y(2), y(3)), pack_bf16x2(y(4), y(5)),
+                                     pack_bf16x2(y(6), y(7)));
           *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) = w;
         }
         fence_proxy_async_smem();

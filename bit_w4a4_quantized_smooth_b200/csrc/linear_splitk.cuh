@@ -36,6 +36,7 @@ constexpr uint32_t kLsPartBytes = kLsBM * kLsPitch * 4;
 struct LsParams {
   const __nv_bfloat16* bias;
   __nv_bfloat16* Y;
+  float alpha;  // a power of two: the 4-bit product's global scales g_x g_w (1 without them)
   int M, K, N, r;
   int splits;   // CTAs per output tile (cluster size along K)
   int spc;      // FP4 stages (256 columns of K) per CTA
@@ -210,11 +211,11 @@ __global__ void __launch_bounds__(kLsThreads, 1)
               float b[8];
 #pragma unroll
               for (int e = 0; e < 8; ++e) b[e] = p.bias ? __bfloat162float(p.bias[n + e]) : 0.0f;
-              *reinterpret_cast<uint4*>(p.Y + static_cast<size_t>(m) * p.N + n) = make_uint4(
-                  pack_bf16x2(__uint_as_float(v[8 * j]) + b[0], __uint_as_float(v[8 * j + 1]) + b[1]),
-                  pack_bf16x2(__uint_as_float(v[8 * j + 2]) + b[2], __uint_as_float(v[8 * j + 3]) + b[3]),
-                  pack_bf16x2(__uint_as_float(v[8 * j + 4]) + b[4], __uint_as_float(v[8 * j + 5]) + b[5]),
-                  pack_bf16x2(__uint_as_float(v[8 * j + 6]) + b[6], __uint_as_float(v[8 * j + 7]) + b[7]));
+              // alpha is a power of two: acc alpha is exact
+              auto y = [&](int e) { return __fmul_rn(__uint_as_float(v[8 * j + e]), p.alpha) + b[e]; };
+              *reinterpret_cast<uint4*>(p.Y + static_cast<size_t>(m) * p.N + n) =
+                  make_uint4(pack_bf16x2(y(0), y(1)), pack_bf16x2(y(2), y(3)), pack_bf16x2(y(4), y(5)),
+                             pack_bf16x2(y(6), y(7)));
             }
           }
         }
@@ -248,6 +249,10 @@ __global__ void __launch_bounds__(kLsThreads, 1)
         acc.z = __fadd_rn(acc.z, b.z);
         acc.w = __fadd_rn(acc.w, b.w);
       }
+      acc.x = __fmul_rn(acc.x, p.alpha);
+      acc.y = __fmul_rn(acc.y, p.alpha);
+      acc.z = __fmul_rn(acc.z, p.alpha);
+      acc.w = __fmul_rn(acc.w, p.alpha);
       if (p.bias) {
         acc.x = __fadd_rn(acc.x, __bfloat162float(p.bias[n]));
         acc.y = __fadd_rn(acc.y, __bfloat162float(p.bias[n + 1]));

@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cmath>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -220,8 +221,8 @@ QaPlan qa_plan(int64_t M, int64_t K, int sms) {
 // reduction), the smaller split on ties.
 svdq_status launch_linear_splitk(const CUtensorMap& tm_xc, const CUtensorMap& tm_rc, const CUtensorMap& tm_xs,
                                  const CUtensorMap& tm_rs, const CUtensorMap& tm_t, const CUtensorMap& tm_l2,
-                                 const void* bias, void* Y, int64_t M, int64_t K, int64_t N, int64_t r, int dev,
-                                 int sms, void* stream) {
+                                 const void* bias, void* Y, int64_t M, int64_t K, int64_t N, int64_t r, float alpha,
+                                 int dev, int sms, void* stream) {
   const int64_t tiles_m = (M + svdq::kLsBM - 1) / svdq::kLsBM;
   const int64_t tiles_n = (N + svdq::kLsBN - 1) / svdq::kLsBN;
   const int64_t tiles = tiles_m * tiles_n;
@@ -253,6 +254,7 @@ svdq_status launch_linear_splitk(const CUtensorMap& tm_xc, const CUtensorMap& tm
   svdq::LsParams p;
   p.bias = static_cast<const __nv_bfloat16*>(bias);
   p.Y = static_cast<__nv_bfloat16*>(Y);
+  p.alpha = alpha;
   p.M = static_cast<int>(M);
   p.K = static_cast<int>(K);
   p.N = static_cast<int>(N);
@@ -435,6 +437,17 @@ svdq_status svdq_quantize_act(const void* X, const float* inv_lambda, const void
 svdq_status svdq_linear(const uint8_t* x_codes, const uint8_t* x_scales, const void* T, const uint8_t* r_codes,
                         const uint8_t* r_scales, const void* L2, const void* bias, int64_t M, int64_t K, int64_t N,
                         int64_t r, void* Y, void* stream) {
+  return svdq_linear_scaled(x_codes, x_scales, T, r_codes, r_scales, L2, bias, M, K, N, r, 1.0f, Y, stream);
+}
+
+svdq_status svdq_linear_scaled(const uint8_t* x_codes, const uint8_t* x_scales, const void* T,
+                               const uint8_t* r_codes, const uint8_t* r_scales, const void* L2, const void* bias,
+                               int64_t M, int64_t K, int64_t N, int64_t r, float alpha, void* Y, void* stream) {
+  // alpha: a power of two in [2^-100, 2^100] (the product acc * alpha is then exact)
+  int alpha_exp = 0;
+  if (!(alpha > 0.0f) || !std::isfinite(alpha) || std::frexp(alpha, &alpha_exp) != 0.5f || alpha_exp < -99 ||
+      alpha_exp > 101)
+    return SVDQ_ERR_INVALID_ARG;
   if (!x_codes || !x_scales || !r_codes || !r_scales || !Y || M <= 0 || K <= 0 || N <= 0)
     return SVDQ_ERR_INVALID_ARG;
   if (r > 0 && (!T || !L2)) return SVDQ_ERR_INVALID_ARG;
@@ -518,9 +531,11 @@ svdq_status svdq_linear(const uint8_t* x_codes, const uint8_t* x_scales, const v
   const int64_t pair_tiles = ((M + svdq::kLinBM - 1) / svdq::kLinBM) * ((N + svdq::kLinBN - 1) / svdq::kLinBN);
   const int path = g_linear_path.load(std::memory_order_relaxed);
   if (path == 2 || (path == 0 && M <= 128 && 4 * pair_tiles < sms))
-    return launch_linear_splitk(tm_xc, tm_rc, tm_xs, tm_rs, tm_t, tm_l2, bias, Y, M, K, N, r, dev, sms, stream);
+    return launch_linear_splitk(tm_xc, tm_rc, tm_xs, tm_rs, tm_t, tm_l2, bias, Y, M, K, N, r, alpha, dev, sms,
+                                stream);
 
   svdq::LinParams p;
+  p.alpha = alpha;
   p.bias = static_cast<const __nv_bfloat16*>(bias);
   p.Y = static_cast<__nv_bfloat16*>(Y);
   p.M = static_cast<int>(M);

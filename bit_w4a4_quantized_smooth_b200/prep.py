@@ -104,3 +104,52 @@ def attach_lora(L1, L2, lam: torch.Tensor, A: torch.Tensor, B: torch.Tensor):
     L1n = LA if L1 is None else torch.cat([L1, LA], dim=1)
     L2n = B if L2 is None else torch.cat([L2, B], dim=0)
     return L1n.contiguous(), L2n.contiguous()
+
+
+# ------------------------------------------------------- global scales ----
+# NVFP4 with a per-tensor global scale g (two-level scaling: a group
+# dequantises to q * decode(s) * g).  g is a power of two chosen so that the
+# tensor's largest group lands in E4M3's top binade: small groups then keep
+# normal (not subnormal or zero) scales, and groups above 6 * 448 no longer
+# saturate.  With powers of two the two-level encoding of Z is the plain
+# encoding of Z / g, so the library's calls take pre-scaled operands
+# (include/svdq.h, svdq_linear_scaled).
+
+E4M3_MAX = 448.0
+
+
+def global_scale(amax: float) -> float:
+    """The power of two 2^ceil(log2(amax / (6 * 448))) (1 for amax = 0)."""
+    import math
+    amax = float(amax)
+    if not (amax > 0.0) or not math.isfinite(amax):
+        return 1.0
+    m, e = math.frexp(amax / (6.0 * E4M3_MAX))  # amax / 2688 = m 2^e, m in [0.5, 1)
+    return math.ldexp(1.0, e if m > 0.5 else e - 1)
+
+
+def _exact_scale(t: torch.Tensor, f: float, name: str) -> torch.Tensor:
+    out = (t.float() * f).to(t.dtype)
+    if not torch.equal((out.float() / f).to(t.dtype), t):
+        raise ValueError(f"{name}: scaling by {f} is not exact (under- or overflow)")
+    return out
+
+
+def apply_global_scales(inv_lambda: torch.Tensor, L2, R: torch.Tensor, gx: float, gw: float):
+    """Operands of the two-level layer for the plain calls:
+    -> (inv_lambda / g_x, L2 / g_w or None, R / g_w, alpha = g_x g_w).
+    Every product is exact (checked: a power of two that under- or
+    overflows raises)."""
+    for g in (gx, gw):
+        import math
+        if not (g > 0.0) or math.frexp(g)[0] != 0.5:
+            raise ValueError(f"global scale {g} is not a power of two")
+    inv_s = _exact_scale(inv_lambda, 1.0 / gx, "inv_lambda")
+    L2_s = None if L2 is None else _exact_scale(L2, 1.0 / gw, "L2")
+    R_s = _exact_scale(R, 1.0 / gw, "R")
+    return inv_s, L2_s, R_s, gx * gw
+
+
+def activation_global_scale(x_amax: torch.Tensor, inv_lambda: torch.Tensor) -> float:
+    """g_x from calibration statistics: the largest |Xh| = max_k amax_k inv_lambda_k."""
+    return global_scale(float((x_amax.float() * inv_lambda.float()).max()))

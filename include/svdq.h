@@ -145,6 +145,28 @@ svdq_status svdq_linear(const uint8_t* x_codes, const uint8_t* x_scales, const v
                         void* stream);
 
 /*
+ * NVFP4 with per-tensor global scales (the NVFP4 format named by the
+ * taicenter.com article on Han Song's team and FLUX carries an fp32 scale per
+ * tensor above the per-16 E4M3 scales).  With global scales g_x for Xh and
+ * g_w for R, a group encodes as s = E4M3_RNE_satfinite(RN_f32(s_f / g)) and
+ * dequantises to q * decode(s) * g, and the layer is
+ *     Y = g_x g_w deq(x) deq(R)^T + T L2 + bias.
+ * For powers of two g this encoding of Z is exactly the plain encoding of
+ * Z / g, so the plain calls serve it on pre-scaled operands:
+ *   svdq_quantize_act with inv_lambda / g_x  -> x codes, scales, and T / g_x
+ *   svdq_pack_residual of R / g_w            -> r codes, scales
+ *   svdq_linear_scaled with L2 / g_w and alpha = g_x g_w
+ * (every pre-scale is exact).  svdq_linear_scaled is svdq_linear with the
+ * accumulator multiplied by alpha before the bias is added:
+ *     Y = bf16(acc * alpha + bias),
+ * alpha a power of two in [2^-100, 2^100] (SVDQ_ERR_INVALID_ARG otherwise),
+ * so the product is exact; alpha = 1 is svdq_linear.
+ */
+svdq_status svdq_linear_scaled(const uint8_t* x_codes, const uint8_t* x_scales, const void* T,
+                               const uint8_t* r_codes, const uint8_t* r_scales, const void* L2, const void* bias,
+                               int64_t M, int64_t K, int64_t N, int64_t r, float alpha, void* Y, void* stream);
+
+/*
  * LoRA adapter joined to the low-rank branch, on the device (chattools.cn
  * article 584, "main functions", item LoRA integration: adapters apply to
  * the quantised model without re-quantising it).  With Xh = X

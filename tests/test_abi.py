@@ -138,3 +138,27 @@ def test_channel_absmax_validation(lib):
     assert f(P(FAKE), 4, 60, P(FAKE), None) == 2         # K not a multiple of 8
     assert f(P(FAKE + 4), 4, 64, P(FAKE), None) == 3     # misaligned X
     assert f(P(FAKE), 4, 64, P(FAKE + 8), None) == 3     # misaligned amax
+
+
+def test_linear_scaled_alpha_validation(lib):
+    P = ctypes.c_void_p
+    f = lib.svdq_linear_scaled
+    f.argtypes = [P, P, P, P, P, P, P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                  ctypes.c_float, P, P]
+    args = [P(FAKE)] * 6 + [None, 128, 256, 256, 32]
+    for bad in (0.0, -2.0, 3.0, 0.3, float("inf"), float("nan"), 2.0 ** -110, 2.0 ** 110):
+        assert f(*args, bad, P(FAKE), None) == 1, bad   # SVDQ_ERR_INVALID_ARG before any launch
+    # a power of two passes the alpha check and fails later on the shape (K % 64)
+    args_bad_k = [P(FAKE)] * 6 + [None, 128, 250, 256, 32]
+    assert f(*args_bad_k, 0.5, P(FAKE), None) == 2
+
+
+def test_global_scale_helpers():
+    import math
+    from bit_w4a4_quantized_smooth_b200 import prep
+    assert prep.global_scale(0.0) == 1.0
+    for amax in (1e-6, 0.37, 1.0, 2688.0, 2688.5, 1e5):
+        g = prep.global_scale(amax)
+        assert math.frexp(g)[0] == 0.5                     # a power of two
+        s = amax / (6.0 * g)                               # the largest group's scale
+        assert 224.0 < s <= 448.0, (amax, g, s)
