@@ -190,10 +190,9 @@ def setup_layer(name: str, device, M=None):
     bias = None if li.bias is None else bf16(li.bias)
     lam, inv = prep.smoothing(X, W)
     L1, L2, R = prep.lowrank(W, lam, li.r)
-    del W
     rc, rs = svdq.pack_residual(R)
     torch.cuda.synchronize()
-    return dict(li=li, X=X, inv=inv, L1=L1, L2=L2, R=R, bias=bias, rc=rc, rs=rs,
+    return dict(li=li, X=X, W=W, inv=inv, L1=L1, L2=L2, R=R, bias=bias, rc=rc, rs=rs,
                 M=li.M, K=li.K, N=li.N, r=li.r)
 
 
@@ -246,10 +245,12 @@ def oracle_sample(X_bits, inv, L1_bits, L2_bits, R, bias_bits, M, K, N, r, targe
     import oracle
     rc, rs = oracle.pack_residual(R)  # per-weight preparation, not timed
 
+    out = {}
+
     def run(rows):
         t0 = time.perf_counter()
         xc, xs, T = oracle.quantize_act(X_bits[:rows], inv, L1_bits, r)
-        oracle.linear_rows(xc, xs, T, rc, rs, L2_bits, bias_bits, rows, K, N, r, np.arange(rows))
+        out["Y"] = oracle.linear_rows(xc, xs, T, rc, rs, L2_bits, bias_bits, rows, K, N, r, np.arange(rows))
         return time.perf_counter() - t0
 
     # grow the sample until it takes about target_s (small samples leave most
@@ -261,7 +262,42 @@ def oracle_sample(X_bits, inv, L1_bits, L2_bits, R, bias_bits, M, K, N, r, targe
             break
         rows = int(max(rows + 1, min(M, rows * 0.9 * target_s / max(t, 1e-3))))
         t = run(rows)
-    return layer_flops(rows, K, N, r) / t / 1e12, rows, t, oracle.num_threads()
+    return layer_flops(rows, K, N, r) / t / 1e12, rows, t, oracle.num_threads(), out["Y"]
+
+
+def rel_err(Y, ref) -> float:
+    """Relative Frobenius error of Y against ref (fp64 host arrays or device tensors)."""
+    import torch
+    if isinstance(Y, torch.Tensor):
+        Y = Y.double()
+        ref = ref.double()
+        return float(torch.linalg.norm(Y - ref) / torch.linalg.norm(ref))
+    return float(np.linalg.norm(Y - ref) / np.linalg.norm(ref))
+
+
+def quality_stats(L, Y):
+    """The layer's quantisation error against the unquantised product X W +
+    bias (fp32 device matmul of the bf16 operands, a statistic only), for the
+    output `Y` of the timed path and for the same layer with per-tensor
+    global scales (NVFP4 two-level scaling)."""
+    import torch
+    import bit_w4a4_quantized_smooth_b200 as svdq
+    from bit_w4a4_quantized_smooth_b200 import prep
+    X, W, bias = L["X"], L["W"], L["bias"]
+    ref = X.float() @ W.float()
+    if bias is not None:
+        ref += bias.float()[None, :]
+    out = {"reference": "unquantised X W + bias, fp32 device matmul of the bf16 operands",
+           "rel_err_gpu": round(rel_err(Y, ref), 5)}
+    gx = prep.activation_global_scale(X.abs().amax(dim=0).float(), L["inv"])
+    gw = prep.global_scale(float(L["R"].abs().max()))
+    inv_s, L2_s, R_s, alpha = prep.apply_global_scales(L["inv"], L["L2"], L["R"], gx, gw)
+    rc, rs = svdq.pack_residual(R_s)
+    xc, xs, T = svdq.quantize_act(X, inv_s, L["L1"])
+    Yg = svdq.linear(xc, xs, T, rc, rs, L2_s, bias, L["M"], L["K"], L["N"], alpha=alpha)
+    out["rel_err_gpu_global_scale"] = round(rel_err(Yg, ref), 5)
+    out["global_scales"] = {"g_x": gx, "g_w": gw}
+    return out, ref
 
 
 # ------------------------------------------------------------- our arm ---
@@ -478,6 +514,12 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
     }
+    # quality statistic, outside every timed region: the timed path's Y
+    # (recomputed: the r = 0 loop above overwrote the buffer) against the
+    # unquantised product
+    step()
+    torch.cuda.synchronize()
+    out["quality"], L["quality_ref"] = quality_stats(L, Y)
     return out, L
 
 
@@ -508,12 +550,16 @@ def main():
             li = L["li"]
             to_np = lambda t: None if t is None else t.detach().cpu().contiguous()
             bits = lambda t: None if t is None else to_np(t).view(torch.int16).numpy().view(np.uint16)
-            v, rows, secs, thr = oracle_sample(li.X, to_np(L["inv"]).numpy(), bits(L["L1"]),
-                                               bits(L["L2"]), to_np(L["R"]).numpy(), li.bias,
-                                               L["M"], L["K"], L["N"], L["r"], args.cpu_seconds)
+            v, rows, secs, thr, Yo = oracle_sample(li.X, to_np(L["inv"]).numpy(), bits(L["L1"]),
+                                                   bits(L["L2"]), to_np(L["R"]).numpy(), li.bias,
+                                                   L["M"], L["K"], L["N"], L["r"], args.cpu_seconds)
             out["cpu_baseline"] = {"value": round(v, 6), "unit": UNIT, "cores": thr, "kind": "oracle",
                                    "sample": f"{rows} of {L['M']} rows (activation step + linear), "
                                              f"{secs:.1f} s, fp64 OpenMP"}
+            if "quality" in out:
+                ref = L["quality_ref"][:rows].double().cpu().numpy()
+                out["quality"]["rel_err_oracle"] = round(rel_err(Yo, ref), 5)
+                out["quality"]["oracle_rows"] = rows
         if world == 1 and not args.no_stack:
             # the whole synthetic DiT stack, one CUDA graph per pass (3 s of
             # preparation on the device, well under a second of timing)
