@@ -83,6 +83,7 @@ def lib() -> ctypes.CDLL:
             ("oracle_dequant", [_P, _P, _I64, _I64, _P]),
             ("oracle_linear_rows", [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _I64, _P]),
             ("oracle_quantize_group_gs", [_P, ctypes.c_float, _P, _P]),
+            ("oracle_quantize_act_ex", [_P, _P, _P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_float, _P, _P, _P]),
             ("oracle_quantize_rows_gs", [_P, _I64, _I64, ctypes.c_float, _P, _P]),
             ("oracle_pack_residual_gs", [_P, _I64, _I64, ctypes.c_float, _P, _P]),
             ("oracle_quantize_act_gs", [_P, _P, _P, _I64, _I64, _I64, ctypes.c_float, _P, _P, _P]),
@@ -93,6 +94,8 @@ def lib() -> ctypes.CDLL:
             f.restype = ctypes.c_int
             f.argtypes = args
         L.oracle_num_threads.restype = ctypes.c_int
+        L.oracle_gelu.restype = ctypes.c_float
+        L.oracle_gelu.argtypes = [ctypes.c_float]
         _lib = L
     return _lib
 
@@ -298,6 +301,25 @@ def quantize_act_gs(X: np.ndarray, inv_lambda: np.ndarray, L1: Optional[np.ndarr
     L1c = None if r == 0 else np.ascontiguousarray(L1, dtype=np.uint16)
     _check(lib().oracle_quantize_act_gs(_ptr(X), _ptr(inv_lambda), _ptr(L1c), M, K, r, float(gx), _ptr(codes),
                                         _ptr(scales), _ptr(T)), "quantize_act_gs")
+    return codes, scales, T
+
+
+def gelu(x: float) -> float:
+    """GELU by Abramowitz and Stegun 7.1.28 in fp32 (the fused activation's rule)."""
+    return lib().oracle_gelu(x)
+
+
+def quantize_act_gelu(X: np.ndarray, inv_lambda: np.ndarray, L1: Optional[np.ndarray], r: int, gx: float = 0.0):
+    """The activation step on GELU(X): Xh = RN_f32(GELU(x) * inv_lambda)."""
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    inv_lambda = np.ascontiguousarray(inv_lambda, dtype=np.float32)
+    M, K = X.shape
+    codes = np.zeros((M, K // 2), dtype=np.uint8)
+    scales = np.zeros(scale_bytes(M, K), dtype=np.uint8)
+    T = np.zeros((M, r), dtype=np.uint16) if r > 0 else None
+    L1c = None if r == 0 else np.ascontiguousarray(L1, dtype=np.uint16)
+    _check(lib().oracle_quantize_act_ex(_ptr(X), _ptr(inv_lambda), _ptr(L1c), M, K, r, 1, float(gx), _ptr(codes),
+                                        _ptr(scales), _ptr(T)), "quantize_act_gelu")
     return codes, scales, T
 
 

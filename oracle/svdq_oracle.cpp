@@ -144,6 +144,44 @@ void quantize_group(const float* v, int64_t stride, uint8_t* codes, uint8_t* sca
   *scale = s;
 }
 
+// ------------------------------------------------------------------ GELU ----
+// GELU(x) = x Phi(x) = 0.5 x (1 + erf(x / sqrt 2)), with erf from the purely
+// rational approximation of Abramowitz and Stegun, Handbook of Mathematical
+// Functions, formula 7.1.28 (|error| <= 3e-7 for x >= 0; erf is odd):
+//   erf(z) ~ 1 - 1 / (1 + a1 z + a2 z^2 + a3 z^3 + a4 z^4 + a5 z^5 + a6 z^6)^16.
+// Every step is one fp32 operation rounded to nearest (no fused multiply-add;
+// this file is built with -ffp-contract=off), in this order:
+//   z = |x| * RN(1/sqrt 2);  p = 1 + z(a1 + z(a2 + z(a3 + z(a4 + z(a5 + z a6)))))
+//   (Horner, a multiply then an add per step);  p16 = (((p^2)^2)^2)^2;
+//   e = 1 - 1/p16;  erf = e with the sign of x;  GELU = (0.5 x) (1 + erf).
+constexpr float kAsA1 = 0.0705230784f, kAsA2 = 0.0422820123f, kAsA3 = 0.0092705272f;
+constexpr float kAsA4 = 0.0001520143f, kAsA5 = 0.0002765672f, kAsA6 = 0.0000430638f;
+constexpr float kRsqrt2 = 0.70710678118654752f;
+
+float gelu_as(float x) {
+  const float z = std::fabs(x) * kRsqrt2;
+  float p = kAsA6;
+  p = p * z;
+  p = p + kAsA5;
+  p = p * z;
+  p = p + kAsA4;
+  p = p * z;
+  p = p + kAsA3;
+  p = p * z;
+  p = p + kAsA2;
+  p = p * z;
+  p = p + kAsA1;
+  p = p * z;
+  p = p + 1.0f;
+  p = p * p;
+  p = p * p;
+  p = p * p;
+  p = p * p;
+  const float e = 1.0f - 1.0f / p;
+  const float erf = std::signbit(x) ? -e : e;
+  return (0.5f * x) * (1.0f + erf);
+}
+
 // ---------------------------------- NVFP4 with a per-tensor global scale ----
 // Two-level scaling: the tensor carries one fp32 scale g > 0 on top of the
 // per-16 E4M3 scales, and an element dequantises to q * decode(s) * g.  One
@@ -440,6 +478,8 @@ int oracle_quantize_rows(const float* V, int64_t rows, int64_t K, uint8_t* codes
   return 0;
 }
 
+float oracle_gelu(float x) { return gelu_as(x); }
+
 // One group of 16 with the two-level quantiser (global scale g > 0).
 int oracle_quantize_group_gs(const float* v, float g, uint8_t* codes, uint8_t* scale) {
   if (!(g > 0.0f)) return 1;
@@ -638,23 +678,36 @@ int oracle_attach_lora(const uint16_t* L1, const uint16_t* L2, const float* lamb
 //   Xh  = RN_f32(X * inv_lambda)             per element
 //   (x_codes, x_scales) = NVFP4(Xh) by groups of 16 along K
 //   T   = bf16(sum_k bf16(Xh)_k L1[k][:])    fp64 sum, one rounding
-int oracle_quantize_act_gs(const uint16_t* X, const float* inv_lambda, const uint16_t* L1, int64_t M,
-                           int64_t K, int64_t r, float gx, uint8_t* x_codes, uint8_t* x_scales, uint16_t* T);
+int oracle_quantize_act_ex(const uint16_t* X, const float* inv_lambda, const uint16_t* L1, int64_t M,
+                           int64_t K, int64_t r, int act, float gx, uint8_t* x_codes, uint8_t* x_scales,
+                           uint16_t* T);
 
 int oracle_quantize_act(const uint16_t* X, const float* inv_lambda, const uint16_t* L1, int64_t M,
                         int64_t K, int64_t r, uint8_t* x_codes, uint8_t* x_scales, uint16_t* T) {
-  return oracle_quantize_act_gs(X, inv_lambda, L1, M, K, r, 0.0f, x_codes, x_scales, T);
+  return oracle_quantize_act_ex(X, inv_lambda, L1, M, K, r, 0, 0.0f, x_codes, x_scales, T);
 }
 
 // The activation step with a global scale g_x for Xh (g_x = 0: the plain
 // quantiser); T is of Xh itself, unaffected by the global scale.
 int oracle_quantize_act_gs(const uint16_t* X, const float* inv_lambda, const uint16_t* L1, int64_t M,
                            int64_t K, int64_t r, float gx, uint8_t* x_codes, uint8_t* x_scales, uint16_t* T) {
-  if (K % 64 != 0 || M < 0 || gx < 0.0f) return 1;
+  return oracle_quantize_act_ex(X, inv_lambda, L1, M, K, r, 0, gx, x_codes, x_scales, T);
+}
+
+// The general form: act = 1 applies GELU (gelu_as, in fp32, no bf16 rounding
+// between) to the input before smoothing, Xh = RN_f32(GELU(x) * inv_lambda);
+// act = 0 is the layer's own activation step.
+int oracle_quantize_act_ex(const uint16_t* X, const float* inv_lambda, const uint16_t* L1, int64_t M,
+                           int64_t K, int64_t r, int act, float gx, uint8_t* x_codes, uint8_t* x_scales,
+                           uint16_t* T) {
+  if (K % 64 != 0 || M < 0 || gx < 0.0f || act < 0 || act > 1) return 1;
   std::vector<float> Xh(static_cast<size_t>(M) * K);
 #pragma omp parallel for schedule(static)
   for (int64_t i = 0; i < M; ++i)
-    for (int64_t k = 0; k < K; ++k) Xh[i * K + k] = bf16_to_f32(X[i * K + k]) * inv_lambda[k];
+    for (int64_t k = 0; k < K; ++k) {
+      const float x = bf16_to_f32(X[i * K + k]);
+      Xh[i * K + k] = (act == 1 ? gelu_as(x) : x) * inv_lambda[k];
+    }
   quantize_rows(Xh.data(), M, K, K, 1, x_codes, x_scales, gx);
   if (r > 0) {
 #pragma omp parallel for schedule(static)
