@@ -68,6 +68,8 @@ def load() -> ctypes.CDLL:
         L.svdq_attach_lora.argtypes = [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P]
         L.svdq_set_linear_path.restype = ctypes.c_int
         L.svdq_set_linear_path.argtypes = [ctypes.c_int]
+        L.svdq_quantize_act_gelu.restype = ctypes.c_int
+        L.svdq_quantize_act_gelu.argtypes = [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, ctypes.c_size_t, _P]
         L.svdq_linear_scaled.restype = ctypes.c_int
         L.svdq_linear_scaled.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_float,
                                          _P, _P]
@@ -143,11 +145,13 @@ def workspace(nbytes: int, device, stream=None):
     return ws
 
 
-def quantize_act(X, inv_lambda, L1, x_codes=None, x_scales=None, T=None, stream=None, workspace_buf=None):
+def quantize_act(X, inv_lambda, L1, x_codes=None, x_scales=None, T=None, stream=None, workspace_buf=None,
+                 gelu: bool = False):
     """X bf16 [M][K], inv_lambda fp32 [K], L1 bf16 [K][r] or None ->
     (x_codes uint8 [M][K/2], x_scales uint8 tiled, T bf16 [M][r] or None).
     The scratch the call needs comes from `workspace_buf` (zero-filled before
-    its first use) or from the binding's per-stream buffer."""
+    its first use) or from the binding's per-stream buffer.  gelu=True runs
+    svdq_quantize_act_gelu (GELU applied to X before smoothing)."""
     import torch
     M, K = X.shape
     r = 0 if L1 is None else L1.shape[1]
@@ -160,9 +164,10 @@ def quantize_act(X, inv_lambda, L1, x_codes=None, x_scales=None, T=None, stream=
         T = torch.empty((M, r), dtype=torch.bfloat16, device=X.device)
     need = quantize_act_workspace_bytes(M, K, r)
     ws = workspace_buf if workspace_buf is not None else workspace(need, X.device, stream)
-    _check(load().svdq_quantize_act(_ptr(X), _ptr(inv_lambda), _ptr(L1), M, K, r, _ptr(x_codes),
-                                    _ptr(x_scales), _ptr(T), _ptr(ws), 0 if ws is None else ws.numel(),
-                                    _stream(stream)), "svdq_quantize_act")
+    fn = load().svdq_quantize_act_gelu if gelu else load().svdq_quantize_act
+    _check(fn(_ptr(X), _ptr(inv_lambda), _ptr(L1), M, K, r, _ptr(x_codes), _ptr(x_scales), _ptr(T), _ptr(ws),
+              0 if ws is None else ws.numel(), _stream(stream)),
+           "svdq_quantize_act_gelu" if gelu else "svdq_quantize_act")
     return x_codes, x_scales, T
 
 

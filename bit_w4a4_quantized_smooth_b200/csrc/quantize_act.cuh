@@ -95,6 +95,35 @@ __host__ __device__ constexpr size_t qa_workspace_bytes(int64_t row_tiles, int s
              : 0;
 }
 
+// GELU(x) = 0.5 x (1 + erf(x / sqrt 2)), erf from the purely rational
+// approximation of Abramowitz and Stegun, Handbook of Mathematical Functions,
+// formula 7.1.28:  erf(z) ~ 1 - (1 + a1 z + ... + a6 z^6)^-16  (z >= 0, odd
+// in z; |error| <= 3e-7 in exact arithmetic).  Evaluated with one rounded fp32
+// operation per step, no fused multiply-add, in a fixed order, so that the
+// result is reproducible bit for bit: z = |x| RN(1/sqrt 2); Horner from a6;
+// four squarings; e = 1 - 1/p16; sign of x; (0.5 x) (1 + erf).
+__device__ __forceinline__ float gelu_as(float x) {
+  const float z = __fmul_rn(fabsf(x), 0.70710678118654752f);
+  float p = 0.0000430638f;
+  p = __fadd_rn(__fmul_rn(p, z), 0.0002765672f);
+  p = __fadd_rn(__fmul_rn(p, z), 0.0001520143f);
+  p = __fadd_rn(__fmul_rn(p, z), 0.0092705272f);
+  p = __fadd_rn(__fmul_rn(p, z), 0.0422820123f);
+  p = __fadd_rn(__fmul_rn(p, z), 0.0705230784f);
+  p = __fadd_rn(__fmul_rn(p, z), 1.0f);
+  p = __fmul_rn(p, p);
+  p = __fmul_rn(p, p);
+  p = __fmul_rn(p, p);
+  p = __fmul_rn(p, p);
+  const float e = __fsub_rn(1.0f, __fdiv_rn(1.0f, p));
+  const float erf = signbit(x) ? -e : e;
+  return __fmul_rn(__fmul_rn(0.5f, x), __fadd_rn(1.0f, erf));
+}
+
+// GELU: the input goes through gelu_as (in fp32, no bf16 rounding between)
+// before the smoothing multiply, Xh = RN_f32(GELU(x) inv_lambda): the MLP's
+// activation fused with the next layer's quantisation.
+template <bool GELU>
 __global__ void __launch_bounds__(kQaThreads, 1)
     quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1,
                         const __grid_constant__ CUtensorMap tm_xc, const QaParams p) {
@@ -288,14 +317,24 @@ __global__ void __launch_bounds__(kQaThreads, 1)
       const float4* lam = reinterpret_cast<const float4*>(stage + lam_off) + 4 * g;
       const float4 l0 = lam[0], l1 = lam[1], l2 = lam[2], l3 = lam[3];
       float v[16];
-      mul2_rn(v[0], v[1], bf16_lo(x0.x), bf16_hi(x0.x), l0.x, l0.y);
-      mul2_rn(v[2], v[3], bf16_lo(x0.y), bf16_hi(x0.y), l0.z, l0.w);
-      mul2_rn(v[4], v[5], bf16_lo(x0.z), bf16_hi(x0.z), l1.x, l1.y);
-      mul2_rn(v[6], v[7], bf16_lo(x0.w), bf16_hi(x0.w), l1.z, l1.w);
-      mul2_rn(v[8], v[9], bf16_lo(x1.x), bf16_hi(x1.x), l2.x, l2.y);
-      mul2_rn(v[10], v[11], bf16_lo(x1.y), bf16_hi(x1.y), l2.z, l2.w);
-      mul2_rn(v[12], v[13], bf16_lo(x1.z), bf16_hi(x1.z), l3.x, l3.y);
-      mul2_rn(v[14], v[15], bf16_lo(x1.w), bf16_hi(x1.w), l3.z, l3.w);
+      {
+        float xi[16] = {bf16_lo(x0.x), bf16_hi(x0.x), bf16_lo(x0.y), bf16_hi(x0.y),
+                        bf16_lo(x0.z), bf16_hi(x0.z), bf16_lo(x0.w), bf16_hi(x0.w),
+                        bf16_lo(x1.x), bf16_hi(x1.x), bf16_lo(x1.y), bf16_hi(x1.y),
+                        bf16_lo(x1.z), bf16_hi(x1.z), bf16_lo(x1.w), bf16_hi(x1.w)};
+        if constexpr (GELU) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) xi[e] = gelu_as(xi[e]);
+        }
+        mul2_rn(v[0], v[1], xi[0], xi[1], l0.x, l0.y);
+        mul2_rn(v[2], v[3], xi[2], xi[3], l0.z, l0.w);
+        mul2_rn(v[4], v[5], xi[4], xi[5], l1.x, l1.y);
+        mul2_rn(v[6], v[7], xi[6], xi[7], l1.z, l1.w);
+        mul2_rn(v[8], v[9], xi[8], xi[9], l2.x, l2.y);
+        mul2_rn(v[10], v[11], xi[10], xi[11], l2.z, l2.w);
+        mul2_rn(v[12], v[13], xi[12], xi[13], l3.x, l3.y);
+        mul2_rn(v[14], v[15], xi[14], xi[15], l3.z, l3.w);
+      }
       float a0m = fmaxf(fabsf(v[0]), fabsf(v[1])), a1m = fmaxf(fabsf(v[2]), fabsf(v[3]));
       float a2m = fmaxf(fabsf(v[4]), fabsf(v[5])), a3m = fmaxf(fabsf(v[6]), fabsf(v[7]));
       a0m = fmaxf(a0m, fmaxf(fabsf(v[8]), fabsf(v[9])));

@@ -328,9 +328,30 @@ svdq_status svdq_quantize_act_workspace(int64_t M, int64_t K, int64_t r, size_t*
   return SVDQ_OK;
 }
 
+namespace {
+svdq_status quantize_act_impl(const void* X, const float* inv_lambda, const void* L1, int64_t M, int64_t K,
+                              int64_t r, uint8_t* x_codes, uint8_t* x_scales, void* T, void* workspace,
+                              size_t workspace_bytes, void* stream, bool gelu);
+}  // namespace
+
 svdq_status svdq_quantize_act(const void* X, const float* inv_lambda, const void* L1, int64_t M, int64_t K,
                               int64_t r, uint8_t* x_codes, uint8_t* x_scales, void* T, void* workspace,
                               size_t workspace_bytes, void* stream) {
+  return quantize_act_impl(X, inv_lambda, L1, M, K, r, x_codes, x_scales, T, workspace, workspace_bytes, stream,
+                           false);
+}
+
+svdq_status svdq_quantize_act_gelu(const void* X, const float* inv_lambda, const void* L1, int64_t M, int64_t K,
+                                   int64_t r, uint8_t* x_codes, uint8_t* x_scales, void* T, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  return quantize_act_impl(X, inv_lambda, L1, M, K, r, x_codes, x_scales, T, workspace, workspace_bytes, stream,
+                           true);
+}
+
+namespace {
+svdq_status quantize_act_impl(const void* X, const float* inv_lambda, const void* L1, int64_t M, int64_t K,
+                              int64_t r, uint8_t* x_codes, uint8_t* x_scales, void* T, void* workspace,
+                              size_t workspace_bytes, void* stream, bool gelu) {
   if (!X || !inv_lambda || !x_codes || !x_scales || M <= 0 || K <= 0) return SVDQ_ERR_INVALID_ARG;
   if (r > 0 && (!L1 || !T)) return SVDQ_ERR_INVALID_ARG;
   if (K % 64 != 0 || !valid_rank(r) || M > kMaxRows || K > kMaxK) return SVDQ_ERR_UNSUPPORTED_SHAPE;
@@ -366,7 +387,8 @@ svdq_status svdq_quantize_act(const void* X, const float* inv_lambda, const void
   }
   const size_t smem = smem_for_tmem(dev, fixed + static_cast<size_t>(stages) * stage_bytes, tmem_cols);
   if (smem == 0 || smem > svdq::kQaSmemLimit) return SVDQ_ERR_CUDA;
-  const void* kern = reinterpret_cast<const void*>(svdq::quantize_act_kernel);
+  auto kfn = gelu ? svdq::quantize_act_kernel<true> : svdq::quantize_act_kernel<false>;
+  const void* kern = reinterpret_cast<const void*>(kfn);
   if (svdq_status rc = ensure_smem(kern, dev, smem)) return rc;
 
   CUtensorMap tm_x, tm_l1, tm_xc;
@@ -429,10 +451,11 @@ svdq_status svdq_quantize_act(const void* X, const float* inv_lambda, const void
   cfg.blockDim = dim3(svdq::kQaThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = static_cast<cudaStream_t>(stream);
-  if (cudaLaunchKernelEx(&cfg, svdq::quantize_act_kernel, tm_x, tm_l1, tm_xc, p) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, kfn, tm_x, tm_l1, tm_xc, p) != cudaSuccess)
     return SVDQ_ERR_CUDA;
   return launch_status();
 }
+}  // namespace
 
 svdq_status svdq_linear(const uint8_t* x_codes, const uint8_t* x_scales, const void* T, const uint8_t* r_codes,
                         const uint8_t* r_scales, const void* L2, const void* bias, int64_t M, int64_t K, int64_t N,

@@ -128,6 +128,23 @@ svdq_status svdq_quantize_act(const void* X, const float* inv_lambda, const void
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The activation step on GELU inputs: svdq_quantize_act with
+ *     Xh = RN_f32(GELU(x) * inv_lambda),
+ * GELU(x) = 0.5 x (1 + erf(x / sqrt 2)) evaluated in fp32 (no bf16 rounding
+ * between GELU and the smoothing multiply), erf by the purely rational
+ * approximation of Abramowitz and Stegun, Handbook of Mathematical Functions,
+ * 7.1.28 (|error| <= 3e-7; in fp32 about 1.5e-6), one rounded operation per
+ * step in a fixed order so the codes are reproducible bit for bit.  The
+ * MLP's activation then costs no pass of its own over the hidden states
+ * (chattools.cn article 584, "Nunchaku": the low-rank and low-bit kernels
+ * are fused to avoid redundant memory access; here the fusion reaches the
+ * next layer's input).  Arguments, workspace and errors as svdq_quantize_act.
+ */
+svdq_status svdq_quantize_act_gelu(const void* X, const float* inv_lambda, const void* L1, int64_t M,
+                                   int64_t K, int64_t r, uint8_t* x_codes, uint8_t* x_scales, void* T,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Fused 4-bit linear: Y = deq(x) deq(R)^T + T L2 + bias, written as bf16.
  * The block-scaled FP4 product and the rank-r bf16 product accumulate in
  * the same fp32 tensor-memory accumulator; bias is added in fp32 and the
