@@ -390,6 +390,19 @@ def run_ours(args, rank, world, local_rank):
 
     lin_r0_us = time_linear(0) if r else lin_us
 
+    # the activation step with GELU fused (svdq_quantize_act_gelu) on the same X
+    def time_qa_gelu(reps=20):
+        es = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in es:
+            flush_l2()
+            a.record(stream)
+            svdq.quantize_act(X, inv, L1, x_codes=xc, x_scales=xs, T=T, stream=stream, gelu=True)
+            b.record(stream)
+        torch.cuda.synchronize()
+        return 1e3 * statistics.mean(a.elapsed_time(b) for a, b in es)
+
+    qa_gelu_us = time_qa_gelu()
+
     # residual packer, once per weight
     pk = []
     for _ in range(10):
@@ -482,6 +495,7 @@ def run_ours(args, rank, world, local_rank):
         "us_per_layer": round(1e3 * ms_per_step, 2),
         "step_us": step_stats(step_ms),
         "quantize_act_us": round(qa_us, 2),
+        "quantize_act_gelu_us": round(qa_gelu_us, 2),
         "linear_us": round(lin_us, 2),
         "linear_r0_us": round(lin_r0_us, 2),
         "lowrank_overhead": round(lin_us / lin_r0_us - 1.0, 4),
@@ -691,26 +705,44 @@ def stack_shape_counts():
     return counts
 
 
+def is_mlp_down(i: int) -> bool:
+    """Stack layer i is a double-stream block's MLP down-projection."""
+    return i < 76 and i % 4 == 3
+
+
 def prepare_stack(device, M=STACK_M, layer_ids=None):
     """Draw and prepare the layers of the synthetic DiT stack (all 152 by
-    default) on the device, untimed: smoothing on the layer's own
-    activations, rank-32 randomized SVD, the rank-32 LoRA adapter joined to
-    the low-rank branch (effective rank 64, R not re-quantised), R packed to
-    NVFP4."""
+    default) on the device, untimed: smoothing, rank-32 randomized SVD, the
+    rank-32 LoRA adapter joined to the low-rank branch (effective rank 64, R
+    not re-quantised), R packed to NVFP4.  A double-stream block's MLP
+    down-projection that directly follows its up-projection is chained: its
+    input is GELU of the up-projection's output, applied inside its
+    activation step (svdq_quantize_act_gelu), and its smoothing statistics
+    come from that output; every other layer reads its own synthetic
+    activations."""
     import torch
     import bit_w4a4_quantized_smooth_b200 as svdq
     from bit_w4a4_quantized_smooth_b200 import prep
     from svdq_inputs import stack_layer_shapes, torch_gen
     layers = []
     for i in (range(len(stack_layer_shapes())) if layer_ids is None else layer_ids):
-        d = torch_gen.make_stack_layer(i, M, device)
-        lam, inv = prep.smoothing(d["X"], d["W"])
+        chain = is_mlp_down(i) and bool(layers) and layers[-1]["id"] == i - 1
+        d = torch_gen.make_stack_layer(i, M, device, with_x=not chain)
+        if chain:
+            up = layers[-1]
+            xc, xs, T = svdq.quantize_act(up["X"], up["inv"], up["L1"], gelu=up["gelu"])
+            Yup = svdq.linear(xc, xs, T, up["rc"], up["rs"], up["L2"], None, M, up["K"], up["N"])
+            amax = torch.nn.functional.gelu(Yup.float()).abs().amax(dim=0)  # calibration statistic only
+            lam, inv = prep.smoothing_from_stats(amax, d["W"])
+            del xc, xs, T, Yup
+        else:
+            lam, inv = prep.smoothing(d["X"], d["W"])
         L1, L2, R = prep.lowrank_randomized(d["W"], lam, 32, seed=i)
         del d["W"]
         L1, L2 = svdq.attach_lora(L1, L2, lam, d["A"], d["B"])
         rc, rs = svdq.pack_residual(R)
         del R
-        layers.append(dict(X=d["X"], inv=inv, L1=L1, L2=L2, rc=rc, rs=rs, K=d["K"], N=d["N"]))
+        layers.append(dict(id=i, X=d["X"], gelu=chain, inv=inv, L1=L1, L2=L2, rc=rc, rs=rs, K=d["K"], N=d["N"]))
     torch.cuda.synchronize()
     return layers
 
@@ -738,10 +770,15 @@ def stack_pass_fn(layers, device, M=STACK_M, Y_out=None):
         K, N, r = L["K"], L["N"], L["L1"].shape[1]
         views.append((xc[: M * K // 2].view(M, K // 2), xs[: svdq.packed_sizes(M, K)[1]],
                       T[: M * r].view(M, r), Y[: M * N].view(M, N) if Y_out is None else Y_out[len(views)]))
+    # a chained layer reads the previous layer's output (in stream order: the
+    # previous linear has written it, and this layer's activation step reads
+    # it before its own linear overwrites the shared buffer)
+    inputs = [views[j - 1][3] if L["gelu"] else L["X"] for j, L in enumerate(layers)]
 
     def run():
-        for L, (xck, xsk, Tk, Yk) in zip(layers, views):
-            svdq.quantize_act(L["X"], L["inv"], L["L1"], x_codes=xck, x_scales=xsk, T=Tk, workspace_buf=ws)
+        for L, Xk, (xck, xsk, Tk, Yk) in zip(layers, inputs, views):
+            svdq.quantize_act(Xk, L["inv"], L["L1"], x_codes=xck, x_scales=xsk, T=Tk, workspace_buf=ws,
+                              gelu=L["gelu"])
             svdq.linear(xck, xsk, Tk, L["rc"], L["rs"], L["L2"], None, M, L["K"], L["N"], Y=Yk)
     return run
 
@@ -806,7 +843,9 @@ def stack_summary(layers, graph_ms, eager_ms, launches, prep_s, peaks, M=STACK_M
     return {
         "workload": "synthetic 12B DiT stack: 19 double-stream blocks (QKV 3072->9216, out 3072->3072, "
                     "MLP 3072->12288->3072) + 38 single-stream blocks (fused 3072->21504, 15360->3072), "
-                    f"M={M}, rank 32 + LoRA 32 (effective 64), no bias",
+                    f"M={M}, rank 32 + LoRA 32 (effective 64), no bias; each MLP down-projection reads "
+                    "GELU of its up-projection's output (GELU fused into its activation step)",
+        "chained_layers": sum(1 for L in layers if L["gelu"]),
         "layers": len(layers), "ms_per_pass": round(graph_ms, 3), "ms_per_pass_eager": round(eager_ms, 3),
         "tflops": round(flops / (graph_ms * 1e-3) / 1e12, 1),
         "roofline_ms": round(roof, 3), "roofline_frac": round(roof / graph_ms, 4),
@@ -837,7 +876,10 @@ def stack_cpu_baseline(rows=8):
         L1 = np.zeros((K, r), dtype=np.uint16)
         L2 = np.zeros((r, N), dtype=np.uint16)
         t0 = time.perf_counter()
-        xc, xs, T = oracle.quantize_act(li.X[:rows], inv, L1, r)
+        if K == 12288:  # the MLP down-projections: GELU inside the activation step
+            xc, xs, T = oracle.quantize_act_gelu(li.X[:rows], inv, L1, r)
+        else:
+            xc, xs, T = oracle.quantize_act(li.X[:rows], inv, L1, r)
         oracle.linear_rows(xc, xs, T, rc, rs, L2, None, rows, K, N, r, np.arange(rows))
         total_s += (time.perf_counter() - t0) * (STACK_M / rows) * n_layers
     return total_s, oracle.num_threads(), (f"{rows} rows of each of the {len(first)} distinct layer shapes, "

@@ -100,24 +100,29 @@ __host__ __device__ constexpr size_t qa_workspace_bytes(int64_t row_tiles, int s
 // formula 7.1.28:  erf(z) ~ 1 - (1 + a1 z + ... + a6 z^6)^-16  (z >= 0, odd
 // in z; |error| <= 3e-7 in exact arithmetic).  Evaluated with one rounded fp32
 // operation per step, no fused multiply-add, in a fixed order, so that the
-// result is reproducible bit for bit: z = |x| RN(1/sqrt 2); Horner from a6;
-// four squarings; e = 1 - 1/p16; sign of x; (0.5 x) (1 + erf).
-__device__ __forceinline__ float gelu_as(float x) {
-  const float z = __fmul_rn(fabsf(x), 0.70710678118654752f);
-  float p = 0.0000430638f;
-  p = __fadd_rn(__fmul_rn(p, z), 0.0002765672f);
-  p = __fadd_rn(__fmul_rn(p, z), 0.0001520143f);
-  p = __fadd_rn(__fmul_rn(p, z), 0.0092705272f);
-  p = __fadd_rn(__fmul_rn(p, z), 0.0422820123f);
-  p = __fadd_rn(__fmul_rn(p, z), 0.0705230784f);
-  p = __fadd_rn(__fmul_rn(p, z), 1.0f);
-  p = __fmul_rn(p, p);
-  p = __fmul_rn(p, p);
-  p = __fmul_rn(p, p);
-  p = __fmul_rn(p, p);
-  const float e = __fsub_rn(1.0f, __fdiv_rn(1.0f, p));
-  const float erf = signbit(x) ? -e : e;
-  return __fmul_rn(__fmul_rn(0.5f, x), __fadd_rn(1.0f, erf));
+// result is reproducible bit for bit: z = |x| RN(1/sqrt 2); Horner from a6
+// (a multiply, then an add); four squarings; e = 1 - RN(1/p16); sign of x;
+// (0.5 x) (1 + erf).
+// Two elements at a time with packed fp32x2 multiplies and adds (each lane
+// rounded as the scalar operation would be); 1/p16 is the correctly rounded
+// reciprocal, the same value as the IEEE quotient 1/p16.
+__device__ __forceinline__ void gelu_as2(float& x0, float& x1) {
+  float z0, z1, p0 = 0.0000430638f, p1 = 0.0000430638f;
+  mul2_rn(z0, z1, fabsf(x0), fabsf(x1), 0.70710678118654752f, 0.70710678118654752f);
+  const float c[6] = {0.0002765672f, 0.0001520143f, 0.0092705272f, 0.0422820123f, 0.0705230784f, 1.0f};
+#pragma unroll
+  for (int i = 0; i < 6; ++i) {
+    mul2_rn(p0, p1, p0, p1, z0, z1);
+    add2_rn(p0, p1, p0, p1, c[i], c[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) mul2_rn(p0, p1, p0, p1, p0, p1);
+  float e0, e1;
+  add2_rn(e0, e1, 1.0f, 1.0f, -__frcp_rn(p0), -__frcp_rn(p1));
+  float h0, h1, s0, s1;
+  mul2_rn(h0, h1, 0.5f, 0.5f, x0, x1);
+  add2_rn(s0, s1, 1.0f, 1.0f, signbit(x0) ? -e0 : e0, signbit(x1) ? -e1 : e1);
+  mul2_rn(x0, x1, h0, h1, s0, s1);
 }
 
 // GELU: the input goes through gelu_as (in fp32, no bf16 rounding between)
@@ -324,7 +329,7 @@ __global__ void __launch_bounds__(kQaThreads, 1)
                         bf16_lo(x1.z), bf16_hi(x1.z), bf16_lo(x1.w), bf16_hi(x1.w)};
         if constexpr (GELU) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) xi[e] = gelu_as(xi[e]);
+          for (int e = 0; e < 16; e += 2) gelu_as2(xi[e], xi[e + 1]);
         }
         mul2_rn(v[0], v[1], xi[0], xi[1], l0.x, l0.y);
         mul2_rn(v[2], v[3], xi[2], xi[3], l0.z, l0.w);

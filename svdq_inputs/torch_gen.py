@@ -103,15 +103,16 @@ def make_lora(seed: int, K: int, N: int, r_lora: int, device, std: float = 0.01)
     return bf16_from_f64(a), bf16_from_f64(b)
 
 
-def make_stack_layer(layer: int, M: int, device):
+def make_stack_layer(layer: int, M: int, device, with_x: bool = True):
     """Layer ``layer`` of the synthetic DiT stack, as
     ``workloads.make_stack_layer_inputs`` defines it, drawn on ``device``:
-    -> dict(X bf16 [M][K], W bf16 [K][N], A bf16 [K][32], B bf16 [32][N], K, N)."""
+    -> dict(X bf16 [M][K] (None without ``with_x``), W bf16 [K][N],
+    A bf16 [K][32], B bf16 [32][N], K, N)."""
     K, N, kind = stack_layer_shapes()[layer]
     seed = config_seed(5, layer)
     n_out = 31 if kind == "outlier" else 0
     lo, hi = (20.0, 100.0) if kind == "outlier" else (1.0, 1.0)
-    X = make_activation(seed, _S_X, M, K, kind, n_out, lo, hi, device)
+    X = make_activation(seed, _S_X, M, K, kind, n_out, lo, hi, device) if with_x else None
     W = make_weight_gauss(seed, K, N, device)
     A, B = make_lora(seed, K, N, STACK_LORA_RANK, device)
     return dict(X=X, W=W, A=A, B=B, K=K, N=N)

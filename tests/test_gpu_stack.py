@@ -12,11 +12,15 @@ def test_stack_pass_matches_layers_alone():
     import bit_w4a4_quantized_smooth_b200 as svdq
     device = torch.device("cuda", 0)
     M = 200  # two activation row tiles, ragged
-    ids = [3, 0, 77, 1, 76, 2]  # widest K first, then narrower: stale tails must not leak
+    # widest K first, then narrower (stale tails must not leak), and an MLP
+    # pair (2 -> 3): layer 3 reads GELU of layer 2's output
+    ids = [77, 0, 76, 1, 2, 3, 4]
     layers = bench.prepare_stack(device, M=M, layer_ids=ids)
+    assert [L["gelu"] for L in layers] == [False, False, False, False, False, True, False]
     ref = []
     for L in layers:
-        xc, xs, T = svdq.quantize_act(L["X"], L["inv"], L["L1"])
+        X = ref[-1] if L["gelu"] else L["X"]
+        xc, xs, T = svdq.quantize_act(X, L["inv"], L["L1"], gelu=L["gelu"])
         ref.append(svdq.linear(xc, xs, T, L["rc"], L["rs"], L["L2"], None, M, L["K"], L["N"]))
     Y = [torch.full((M, L["N"]), float("nan"), dtype=torch.bfloat16, device=device) for L in layers]
     run = bench.stack_pass_fn(layers, device, M=M, Y_out=Y)
