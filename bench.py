@@ -49,7 +49,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
-    ap.add_argument("--once", choices=["quantize_act", "linear", "pack_residual"],
+    ap.add_argument("--once", choices=["quantize_act", "quantize_act_gelu", "linear", "pack_residual"],
                     help="no timing: three launches of one kernel on the workload (for profilers)")
     ap.add_argument("--rows", type=int, default=None,
                     help="with --once: M rows instead of the workload's (same distributions)")
@@ -67,7 +67,7 @@ def parse_args():
 # `bench.py --once linear --workload <name>` (L2-warm), per workload.  A figure
 # is reported only while the kernel sources hash to the captured ones.
 LINEAR_TRAFFIC_CAPTURES = {
-    "flux_mlp_up": {"bytes": 30408960 + 58434304, "sources_sha256": "36fbc53256e6394a"},
+    "flux_mlp_up": {"bytes": 30390272 + 58081536, "sources_sha256": "fe8ba598e8abb3b2"},
 }
 
 
@@ -605,8 +605,9 @@ def run_once(args):
     xc, xs, T = svdq.quantize_act(L["X"], L["inv"], L["L1"])
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
     for _ in range(3):
-        if args.once == "quantize_act":
-            svdq.quantize_act(L["X"], L["inv"], L["L1"], x_codes=xc, x_scales=xs, T=T)
+        if args.once in ("quantize_act", "quantize_act_gelu"):
+            svdq.quantize_act(L["X"], L["inv"], L["L1"], x_codes=xc, x_scales=xs, T=T,
+                              gelu=args.once == "quantize_act_gelu")
         elif args.once == "linear":
             svdq.linear(xc, xs, T, L["rc"], L["rs"], L["L2"], L["bias"], M, K, N, Y=Y)
         else:
