@@ -11,8 +11,7 @@
 // through a deep shared-memory ring (the ring's depth, not the bandwidth,
 // sets the pace: every slot waits out a loaded TMA latency and a few warp
 // hand-offs before it is refilled):
-//   warp 16     TMA producer: first an L2 prefetch of the CTA's next atoms
-//               (X and L1, a fixed distance ahead); per atom the X tile (128
+//   warp 16     TMA producer: per atom the X tile (128
 //               rows x 64 columns, K-major, 128-byte swizzle), the atom's L1
 //               rows (64 k x 64 or 128 ranks, rank-contiguous, 128-byte
 //               swizzle; ranks past r arrive as zeros) and its 64 inv_lambda;
@@ -52,7 +51,6 @@ constexpr int kQaProducerWarp = 16;
 constexpr int kQaMmaWarp = 17;
 constexpr int kQaStoreWarp = 18;
 constexpr int kQaThreads = 19 * 32;
-constexpr int kQaPrefetch = 16;              // atoms the L2 prefetch runs ahead
 constexpr int kQaMaxStages = 8;
 constexpr int kQaMaxSplits = 16;
 constexpr uint32_t kQaXBytes = kQaRows * 128;  // one X atom
@@ -197,12 +195,10 @@ __global__ void __launch_bounds__(kQaThreads, 1)
       if (has_lr) prefetch_tmap(&tm_l1);
     }
     __syncwarp();
-    const int pf = min(na, kQaPrefetch);
-    for (int c = 0; c < pf; ++c) {
-      const int k = (a0 + c) * 64;
-      e_tma_prefetch_2d(&tm_x, k, row0);
-      for (int t = 0; t < p.n_l1; ++t) e_tma_prefetch_2d(&tm_l1, 64 * t, k);
-    }
+    // No L2 prefetch ahead of the ring: measured on B200, prefetching the
+    // CTA's atoms first delayed the ring's own first loads by about 2 us and
+    // lengthened the stream (4 us at K = 3072, 8 us at K = 12288); the ring's
+    // loads alone keep enough bytes in flight.
     const uint32_t tx = kQaXBytes + l1_bytes + 256u;
     int issued = 0;
     int s = 0;
@@ -220,11 +216,6 @@ __global__ void __launch_bounds__(kQaThreads, 1)
       e_tma_load_2d(dst, &tm_x, fb, k, row0);
       for (int t = 0; t < p.n_l1; ++t) e_tma_load_2d(dst + kQaXBytes + t * kQaL1AtomBytes, &tm_l1, fb, 64 * t, k);
       e_bulk_load(dst + lam_off, p.inv_lambda + k, 256u, fb);
-      if (c + kQaPrefetch < na) {
-        const int kp = k + 64 * kQaPrefetch;
-        e_tma_prefetch_2d(&tm_x, kp, row0);
-        for (int t = 0; t < p.n_l1; ++t) e_tma_prefetch_2d(&tm_l1, 64 * t, kp);
-      }
       ++issued;
       if (++s == S) {
         s = 0;
