@@ -944,9 +944,11 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": dict(workload_desc(args.workload, M, K, N, r), parallelism="cpu"),
+        # the same workload description as our arm's line; where it ran is in cpu_baseline
+        "config": dict(workload_desc(args.workload, M, K, N, r), parallelism=f"replicas{args.gpus}"),
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": oracle.num_threads(),
-                         "kind": "oracle", "sample": f"{rows} of {M} rows per step"},
+                         "kind": "oracle", "device": "host cores (rank 0)",
+                         "sample": f"{rows} of {M} rows per step"},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
