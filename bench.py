@@ -60,6 +60,8 @@ def parse_args():
                          "with the oracle's extrapolated time beside it")
     ap.add_argument("--no-stack", action="store_true",
                     help="leave the DiT stack pass out of the default single-GPU line")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="launch the layer kernels plainly (svdq_set_launch_overlap(0)), for comparison")
     return ap.parse_args()
 
 
@@ -558,6 +560,9 @@ def main():
         return 0
     import torch
     import torch.distributed as dist
+    if args.no_overlap:
+        import bit_w4a4_quantized_smooth_b200 as svdq
+        svdq.set_launch_overlap(False)
     if args.once:
         return run_once(args)
     if args.sweep:
@@ -595,6 +600,7 @@ def main():
             g_ms, e_ms, launches = time_stack(layers, torch.device("cuda", local_rank))
             out["stack"] = stack_summary(layers, g_ms, e_ms, launches, prep_s, load_peaks())
             del layers
+        out["launch_overlap"] = not args.no_overlap
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:
@@ -711,7 +717,7 @@ def run_sweep(args):
                 "algorithmic_gbs": round(nbytes / (us * 1e-6) / 1e9, 1),
                 "bound": "tensor" if flops / (fp4_peak * 1e12) > nbytes / (peaks["hbm_gbs"] * 1e9) else "hbm",
                 "roofline_frac": round(roof_us / us, 4), "reps": reps,
-                "l2": "flushed before every rep"}), flush=True)
+                "l2": "flushed before every rep", "launch_overlap": not args.no_overlap}), flush=True)
     return 0
 
 
@@ -922,6 +928,7 @@ def run_stack(args):
         secs, thr, sample = stack_cpu_baseline()
         out["stack"]["cpu_baseline"] = {"ms_per_pass": round(secs * 1e3, 1), "cores": thr, "kind": "oracle",
                                         "sample": sample}
+    out["launch_overlap"] = not args.no_overlap
     print(json.dumps(out), flush=True)
     return 0
 

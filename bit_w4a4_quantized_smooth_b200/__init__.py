@@ -19,6 +19,7 @@ from .binding import (  # noqa: F401
     packed_sizes,
     quantize_act,
     selftest_wait_timeout,
+    set_launch_overlap,
     set_linear_path,
     set_wait_timeout,
     status_string,

@@ -68,6 +68,8 @@ def load() -> ctypes.CDLL:
         L.svdq_attach_lora.argtypes = [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P]
         L.svdq_set_linear_path.restype = ctypes.c_int
         L.svdq_set_linear_path.argtypes = [ctypes.c_int]
+        L.svdq_set_launch_overlap.restype = ctypes.c_int
+        L.svdq_set_launch_overlap.argtypes = [ctypes.c_int]
         L.svdq_quantize_act_gelu.restype = ctypes.c_int
         L.svdq_quantize_act_gelu.argtypes = [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, ctypes.c_size_t, _P]
         L.svdq_linear_scaled.restype = ctypes.c_int
@@ -256,6 +258,13 @@ LINEAR_PATHS = {"auto": 0, "large": 1, "small": 2}
 def set_linear_path(path: str):
     """Force svdq_linear's kernel: "auto" (by shape), "large" or "small"."""
     _check(load().svdq_set_linear_path(LINEAR_PATHS[path]), "svdq_set_linear_path")
+
+
+def set_launch_overlap(enable: bool):
+    """Whether the layer calls' kernels may start their set-up while the
+    kernel ahead of them in the stream finishes (default True); results are
+    the same either way."""
+    _check(load().svdq_set_launch_overlap(1 if enable else 0), "svdq_set_launch_overlap")
 
 
 def selftest_wait_timeout(timeout_ns: int, stream=None):

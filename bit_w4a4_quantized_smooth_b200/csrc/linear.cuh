@@ -50,6 +50,7 @@ constexpr uint32_t kLinStageOut = kLinStages * kLinStageBytes + 1024;  // after 
 constexpr uint32_t kLinOutBytes = 4096;     // one warp's 32 x 64 bf16 output block
 constexpr uint32_t kLinBarOffset = kLinStageOut + 4 * 2 * kLinOutBytes;  // 2 blocks per epilogue warp
 constexpr int kLinNumBars = 2 * kLinStages + 2 + 2 + 1 + 1 + 1;
+constexpr int kLinWarmStages = 16;  // stages whose weights are prefetched before the wait
 
 struct LinParams {
   const __nv_bfloat16* bias;
@@ -119,6 +120,9 @@ __global__ void __launch_bounds__(kLinThreads, 1)
   __syncthreads();
   cluster_sync();  // the even CTA's barriers exist before anyone signals them
   tc_fence_after();
+  // The next layer's activation step may now be scheduled (after the tensor
+  // memory is held, so that no later CTA can hold it while waiting for us).
+  griddep_launch_dependents();
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(smem);
   auto lead = [&](const uint64_t* bar) { return map_shared_rank(smem_u32(bar), 0); };
@@ -136,6 +140,24 @@ __global__ void __launch_bounds__(kLinThreads, 1)
       }
     }
     __syncwarp();
+    // While the activation step ahead finishes: the weight halves (L2, R
+    // codes and scales) of the first tile's first stages into L2.
+    if (pair < p.tiles) {
+      const int n0 = (pair / p.m_tiles) * kLinBN;
+      const int nb = n0 + 128 * static_cast<int>(rank);
+      for (int it = 0; it < min(total, kLinWarmStages); ++it) {
+        if (it < n_lr) {
+          e_tma_prefetch_2d(&tm_l2, nb, it * 64);
+          e_tma_prefetch_2d(&tm_l2, nb + 64, it * 64);
+        } else {
+          const int kt = (it - n_lr) * (kLinBK / 64);
+          e_tma_prefetch_2d(&tm_rc, kt * 32, nb);
+          e_tma_prefetch_3d(&tm_rs, 0, 0, (n0 >> 7) * tiles_k + kt);
+          e_tma_prefetch_3d(&tm_rs, 0, 0, ((n0 >> 7) + 1) * tiles_k + kt);
+        }
+      }
+    }
+    griddep_wait();
     uint32_t g = 0;
     bool ok = true;
     for (int t = pair; t < p.tiles && ok && !warp_flag(abort_flag); t += pairs) {
@@ -205,6 +227,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
       }
     }
   } else if (warp == 1) {
+    griddep_wait();  // bounded waits start once the kernel ahead is done
     if (rank == 0) {
       // -------------------------------------------------- MMA issuer --
       const uint32_t idesc_f4 = (1u << 7) | (1u << 10) | ((kLinBN >> 3) << 17) | ((kLinBM >> 4) << 24);
@@ -263,6 +286,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     }
   } else {
     // ------------------------------------------------------- epilogue --
+    griddep_wait();            // the bias and Y may belong to the kernel ahead
     const int et = tid - 64;   // 0..127
     const int q = warp & 3;    // TMEM lane quadrant this warp may access
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;

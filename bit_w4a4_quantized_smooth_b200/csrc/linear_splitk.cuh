@@ -32,6 +32,7 @@ constexpr uint32_t kLsTmemCols = 256;       // accumulator [0, 128), scale facto
 constexpr uint32_t kLsSfaCol = 128, kLsSfbCol = 144;
 constexpr int kLsPitch = kLsBN + 4;         // floats per row of a partial (16-byte skew)
 constexpr uint32_t kLsPartBytes = kLsBM * kLsPitch * 4;
+constexpr int kLsWarmStages = 16;           // stages whose weights are prefetched before the wait
 
 struct LsParams {
   const __nv_bfloat16* bias;
@@ -90,6 +91,9 @@ __global__ void __launch_bounds__(kLsThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // The next layer's activation step may now be scheduled (after the tensor
+  // memory is held, so that no later CTA can hold it while waiting for us).
+  griddep_launch_dependents();
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(ring);
 
@@ -106,6 +110,19 @@ __global__ void __launch_bounds__(kLsThreads, 1)
       }
     }
     __syncwarp();
+    // While the activation step ahead finishes: this CTA's weight halves (L2,
+    // R codes and scales) into L2, up to kLsWarmStages stages.
+    for (int it = 0; it < min(total, kLsWarmStages); ++it) {
+      if (it < n_lr) {
+        e_tma_prefetch_2d(&tm_l2, n0, it * 64);
+        e_tma_prefetch_2d(&tm_l2, n0 + 64, it * 64);
+      } else {
+        const int ks = kt0 + it - n_lr;
+        e_tma_prefetch_2d(&tm_rc, ks * 128, n0);
+        e_tma_prefetch_3d(&tm_rs, 0, 0, (n0 >> 7) * tiles_k + 4 * ks);
+      }
+    }
+    griddep_wait();
     int issued = 0;
     for (int it = 0; it < total; ++it) {
       const int s = it % S;
@@ -143,6 +160,7 @@ __global__ void __launch_bounds__(kLsThreads, 1)
         warp_wait(smem_u32(&full[c % S]), (c / S) & 1, p.timeout_ns, 51);
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
+    griddep_wait();  // bounded waits start once the kernel ahead is done
     const uint32_t idesc_f4 = (1u << 7) | (1u << 10) | ((kLsBN >> 3) << 17) | ((kLsBM >> 4) << 24);
     const uint32_t idesc_bf =
         (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((kLsBN >> 3) << 17) | ((kLsBM >> 4) << 24);
@@ -188,6 +206,7 @@ __global__ void __launch_bounds__(kLsThreads, 1)
   }
 
   // --------------------------------------------------------- epilogue --
+  griddep_wait();   // the bias and Y may belong to the kernel ahead
   __syncthreads();  // every role is done: the ring is idle, the MMAs complete
   const bool aborted = *abort_flag != 0;
   float* part = reinterpret_cast<float*>(ring);  // [128][kLsPitch], over the idle ring

@@ -78,6 +78,22 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
   }
 }
 
+// ------------------------------------------- programmatic dependent launch --
+// The layer's kernels are launched with the programmatic stream-serialisation
+// attribute: a grid may be scheduled while the kernel ahead of it in the
+// stream still runs, once every CTA of that kernel has issued
+// griddep_launch_dependents() (or exited).  griddep_wait() returns when the
+// kernel ahead has completed and its memory writes are visible; every thread
+// waits before it touches global memory the kernel ahead may write or read
+// (L2 prefetches excepted: L2 is the device's point of coherence, so a
+// prefetch can fetch a line early but never a stale one).  Without such a
+// predecessor the wait returns at once.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------- TMA --
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
@@ -254,6 +270,14 @@ __device__ __forceinline__ void e_tma_prefetch_2d(const void* tmap, int x, int y
   asm volatile(SVDQ_ELECT_BEGIN "@e cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" SVDQ_ELECT_END ::"l"(
                    tmap),
                "r"(x), "r"(y)
+               : "memory");
+}
+
+// Prefetch a 3-D box of a tensor into L2.
+__device__ __forceinline__ void e_tma_prefetch_3d(const void* tmap, int x, int y, int z) {
+  asm volatile(SVDQ_ELECT_BEGIN "@e cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" SVDQ_ELECT_END ::"l"(
+                   tmap),
+               "r"(x), "r"(y), "r"(z)
                : "memory");
 }
 

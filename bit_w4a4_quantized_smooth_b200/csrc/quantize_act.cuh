@@ -184,6 +184,12 @@ __global__ void __launch_bounds__(kQaThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // The kernel behind this one may now be scheduled; only now, with this
+  // CTA's tensor memory held: a later kernel's CTA that took it first would
+  // wait in its griddep_wait for this grid while this CTA waited for its
+  // tensor memory.
+  griddep_launch_dependents();
+  griddep_wait();  // X, the outputs and the workspace may belong to the kernel ahead
   const uint32_t tmem = has_lr ? *tmem_slot : 0u;
   const uint32_t sbase = smem_u32(ring);
 

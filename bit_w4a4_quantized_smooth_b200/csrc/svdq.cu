@@ -33,6 +33,21 @@ constexpr int64_t kMaxK = int64_t(1) << 20;
 // large-M kernel, 2 the small-M kernel (svdq_set_linear_path).
 std::atomic<int> g_linear_path{0};
 
+// Whether the layer's launches carry the programmatic stream-serialisation
+// attribute (svdq_set_launch_overlap; default on).  With it a layer kernel
+// may be scheduled while the kernel ahead of it in the stream finishes; it
+// sets up (barriers, tensor memory, L2 prefetch of weights) and then waits
+// in-kernel for that kernel before it touches anything it could share with it.
+std::atomic<int> g_overlap{1};
+
+// Appends the overlap attribute to attrs[n] when the setting is on.
+unsigned add_overlap_attr(cudaLaunchAttribute* attrs, unsigned n) {
+  if (!g_overlap.load(std::memory_order_relaxed)) return n;
+  attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[n].val.programmaticStreamSerializationAllowed = 1;
+  return n + 1;
+}
+
 // -------------------------------------------------------- wait timeout --
 std::atomic<uint64_t> g_timeout_ns{0};
 
@@ -268,13 +283,17 @@ svdq_status launch_linear_splitk(const CUtensorMap& tm_xc, const CUtensorMap& tm
   cfg.blockDim = dim3(svdq::kLsThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(splits);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  unsigned na = 0;
+  if (splits > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(splits);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    na = 1;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = splits > 1 ? 1 : 0;
+  cfg.numAttrs = add_overlap_attr(attr, na);
   if (cudaLaunchKernelEx(&cfg, svdq::linear_splitk_kernel, tm_xc, tm_rc, tm_xs, tm_rs, tm_t, tm_l2, p) !=
       cudaSuccess)
     return SVDQ_ERR_CUDA;
@@ -451,6 +470,9 @@ svdq_status quantize_act_impl(const void* X, const float* inv_lambda, const void
   cfg.blockDim = dim3(svdq::kQaThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  cfg.attrs = attr;
+  cfg.numAttrs = add_overlap_attr(attr, 0);
   if (cudaLaunchKernelEx(&cfg, kfn, tm_x, tm_l1, tm_xc, p) != cudaSuccess)
     return SVDQ_ERR_CUDA;
   return launch_status();
@@ -579,13 +601,13 @@ svdq_status svdq_linear_scaled(const uint8_t* x_codes, const uint8_t* x_scales, 
   cfg.blockDim = dim3(svdq::kLinThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = add_overlap_attr(attr, 1);
   if (cudaLaunchKernelEx(&cfg, kern, tm_xc, tm_rc, tm_xs, tm_rs, tm_t, tm_l2, tm_y, p) != cudaSuccess)
     return SVDQ_ERR_CUDA;
   return launch_status();
@@ -666,6 +688,12 @@ svdq_status svdq_set_wait_timeout(uint64_t timeout_ns) {
 svdq_status svdq_set_linear_path(int path) {
   if (path < 0 || path > 2) return SVDQ_ERR_INVALID_ARG;
   g_linear_path.store(path, std::memory_order_relaxed);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_set_launch_overlap(int enable) {
+  if (enable != 0 && enable != 1) return SVDQ_ERR_INVALID_ARG;
+  g_overlap.store(enable, std::memory_order_relaxed);
   return SVDQ_OK;
 }
 

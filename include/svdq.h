@@ -236,6 +236,23 @@ svdq_status svdq_channel_absmax(const void* X, int64_t M, int64_t K, float* amax
 svdq_status svdq_set_linear_path(int path);
 
 /*
+ * Launch overlap of the layer calls (host-side setting for the whole
+ * process; 1 by default).  With 1, svdq_quantize_act(_gelu, _noalloc) and
+ * svdq_linear(_scaled) launch their kernels with CUDA's programmatic
+ * stream-serialisation attribute: a kernel may be scheduled while the
+ * kernel ahead of it in the stream is finishing, sets up (barriers, tensor
+ * memory; the linear kernels also prefetch their weight tiles into L2) and
+ * waits on the device for that kernel to complete before it reads or writes
+ * any buffer.  Stream order is therefore kept for every buffer, whatever
+ * kernel precedes the call; only the set-up overlaps.  The layer kernels in
+ * turn let the kernel behind them start its set-up early.  Inside a CUDA
+ * graph captured from a stream the overlap becomes a programmatic edge.
+ * With 0 the kernels launch plainly.  Results are identical either way.
+ * Returns SVDQ_ERR_INVALID_ARG for values other than 0 and 1.
+ */
+svdq_status svdq_set_launch_overlap(int enable);
+
+/*
  * Failure detection.  Every wait inside the kernels is bounded (default
  * 2 s, or SVDQ_WAIT_TIMEOUT_MS from the environment at first use); a wait
  * that expires records SVDQ_ERR_TIMEOUT in the current device's status word

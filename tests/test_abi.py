@@ -162,3 +162,11 @@ def test_global_scale_helpers():
         assert math.frexp(g)[0] == 0.5                     # a power of two
         s = amax / (6.0 * g)                               # the largest group's scale
         assert 224.0 < s <= 448.0, (amax, g, s)
+
+
+def test_launch_overlap_setting(lib):
+    from bit_w4a4_quantized_smooth_b200 import set_launch_overlap
+    assert lib.svdq_set_launch_overlap(2) == 1      # SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_set_launch_overlap(-1) == 1
+    set_launch_overlap(False)
+    set_launch_overlap(True)                         # the default, restored
