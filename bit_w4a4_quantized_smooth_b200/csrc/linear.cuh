@@ -50,7 +50,6 @@ constexpr uint32_t kLinStageOut = kLinStages * kLinStageBytes + 1024;  // after 
 constexpr uint32_t kLinOutBytes = 4096;     // one warp's 32 x 64 bf16 output block
 constexpr uint32_t kLinBarOffset = kLinStageOut + 4 * 2 * kLinOutBytes;  // 2 blocks per epilogue warp
 constexpr int kLinNumBars = 2 * kLinStages + 2 + 2 + 1 + 1 + 1;
-constexpr int kLinWarmStages = 16;  // stages whose weights are prefetched before the wait
 
 struct LinParams {
   const __nv_bfloat16* bias;
@@ -141,11 +140,13 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     }
     __syncwarp();
     // While the activation step ahead finishes: the weight halves (L2, R
-    // codes and scales) of the first tile's first stages into L2.
+    // codes and scales) of the stages the ring loads first into L2 (measured
+    // on B200, same box: the linear alone 96.2-96.5 us with these five
+    // stages, 96.5-97.2 us with sixteen, 98.3-98.4 us without).
     if (pair < p.tiles) {
       const int n0 = (pair / p.m_tiles) * kLinBN;
       const int nb = n0 + 128 * static_cast<int>(rank);
-      for (int it = 0; it < min(total, kLinWarmStages); ++it) {
+      for (int it = 0; it < min(total, kLinStages); ++it) {
         if (it < n_lr) {
           e_tma_prefetch_2d(&tm_l2, nb, it * 64);
           e_tma_prefetch_2d(&tm_l2, nb + 64, it * 64);

@@ -32,7 +32,6 @@ constexpr uint32_t kLsTmemCols = 256;       // accumulator [0, 128), scale facto
 constexpr uint32_t kLsSfaCol = 128, kLsSfbCol = 144;
 constexpr int kLsPitch = kLsBN + 4;         // floats per row of a partial (16-byte skew)
 constexpr uint32_t kLsPartBytes = kLsBM * kLsPitch * 4;
-constexpr int kLsWarmStages = 16;           // stages whose weights are prefetched before the wait
 
 struct LsParams {
   const __nv_bfloat16* bias;
@@ -110,9 +109,9 @@ __global__ void __launch_bounds__(kLsThreads, 1)
       }
     }
     __syncwarp();
-    // While the activation step ahead finishes: this CTA's weight halves (L2,
-    // R codes and scales) into L2, up to kLsWarmStages stages.
-    for (int it = 0; it < min(total, kLsWarmStages); ++it) {
+    // While the activation step ahead finishes: the weight halves (L2, R
+    // codes and scales) of the stages the ring loads first into L2.
+    for (int it = 0; it < min(total, S); ++it) {
       if (it < n_lr) {
         e_tma_prefetch_2d(&tm_l2, n0, it * 64);
         e_tma_prefetch_2d(&tm_l2, n0 + 64, it * 64);
