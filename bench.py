@@ -109,6 +109,58 @@ def load_peaks():
 FP4_OVER_BF16 = 4.0
 
 
+# ------------------------------------------------ library FP4 reference ---
+
+LIBRARY_FP4_PEAK_SHAPE = (8192, 8192, 8192)
+
+
+def library_fp4_times(device, flush_l2, shapes, reps=20):
+    """Median µs of cuBLASLt's NVFP4 GEMM (torch's block-scaled scaled_mm:
+    E2M1 codes, E4M3 scales per 16 along K in the 128 x 4 tile layout,
+    bf16 output) for each (M, N, K) of `shapes`, on random codes with unit
+    scales and L2 flushed before every rep.  A library-achieved FP4 rate to
+    read the linear kernel against; nothing of the layer's path uses it.
+    -> ({shape: us}, api) or (None, reason) when torch does not expose it."""
+    import torch
+    import bit_w4a4_quantized_smooth_b200 as svdq
+    try:
+        from torch.nn.functional import ScalingType, SwizzleType, scaled_mm
+    except ImportError as e:
+        return None, f"torch.nn.functional.scaled_mm unavailable ({e})"
+    out = {}
+    for (M, N, K) in shapes:
+        g = torch.Generator(device=device)
+        g.manual_seed(0)
+        a = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=device, generator=g)
+        b = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=device, generator=g)
+        sa = torch.full((svdq.packed_sizes(M, K)[1],), 0x38, dtype=torch.uint8, device=device)  # E4M3 1.0
+        sb = torch.full((svdq.packed_sizes(N, K)[1],), 0x38, dtype=torch.uint8, device=device)
+        A, B = a.view(torch.float4_e2m1fn_x2), b.view(torch.float4_e2m1fn_x2).t()
+        SA, SB = sa.view(torch.float8_e4m3fn), sb.view(torch.float8_e4m3fn)
+
+        def fn():
+            return scaled_mm(A, B, SA, ScalingType.BlockWise1x16, SB, ScalingType.BlockWise1x16,
+                             swizzle_a=SwizzleType.SWIZZLE_32_4_4, swizzle_b=SwizzleType.SWIZZLE_32_4_4,
+                             output_dtype=torch.bfloat16)
+        try:
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+        except Exception as e:  # an unsupported build or device
+            return None, f"scaled_mm NVFP4 failed: {type(e).__name__}: {str(e)[:120]}"
+        ev = []
+        for _ in range(reps):
+            flush_l2()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            ev.append((e0, e1))
+        torch.cuda.synchronize()
+        out[(M, N, K)] = statistics.median(1e3 * e0.elapsed_time(e1) for e0, e1 in ev)
+    return out, "torch.nn.functional.scaled_mm, BlockWise1x16 E4M3 scales (cuBLASLt)"
+
+
 # ---------------------------------------------------------------- clocks ---
 
 class ClockSampler:
@@ -540,6 +592,20 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
     }
+    # library-achieved FP4 rate (outside every timed region): cuBLASLt's
+    # NVFP4 GEMM at 8192^3 and on this layer's FP4 product
+    lib, api = library_fp4_times(device, flush_l2, [LIBRARY_FP4_PEAK_SHAPE, (M, N, K)])
+    if lib is None:
+        out["fp4_library"] = {"unavailable": api}
+    else:
+        pm, pn, pk = LIBRARY_FP4_PEAK_SHAPE
+        lib_peak = 2.0 * pm * pn * pk / (lib[LIBRARY_FP4_PEAK_SHAPE] * 1e-6) / 1e12
+        out["fp4_library"] = {
+            "api": api, "peak_shape": f"{pm}x{pn}x{pk}", "peak_tflops": round(lib_peak, 1),
+            "linear_frac": round(achieved / lib_peak, 4),
+            "same_shape_us": round(lib[(M, N, K)], 2),
+            "note": "library-achieved FP4 rate (random codes, unit scales, L2 flushed); the FP4 product "
+                    "only (no low-rank branch, no bias); not on the layer's path"}
     # quality statistic, outside every timed region: the timed path's Y
     # (recomputed: the r = 0 loop above overwrote the buffer) against the
     # unquantised product
