@@ -438,6 +438,16 @@ def run_ours(args, rank, world, local_rank):
     qa_us = 1e3 * statistics.mean(e[0].elapsed_time(e[1]) for e in evk)
     lin_us = 1e3 * statistics.mean(e[1].elapsed_time(e[2]) for e in evk)
 
+    # host cost of one step through the Python binding (argument checks, the
+    # cached tensor maps, the two launches), on the CPU clock while the GPU
+    # runs behind; no flush, nothing synchronised inside the loop
+    host_steps = 50
+    t_host = time.perf_counter()
+    for _ in range(host_steps):
+        step()
+    host_us = (time.perf_counter() - t_host) * 1e6 / host_steps
+    torch.cuda.synchronize()
+
     # plain FP4 GEMM (rank 0 branch switched off) on the same operands, for
     # the low-rank overhead
     def time_linear(rr, reps=20):
@@ -566,6 +576,7 @@ def run_ours(args, rank, world, local_rank):
         "pack_residual_us": round(pack_us, 2),
         "pack_residual_gbs": round((K * N * 4 + N * K // 2 + N * K // 16) / (pack_us * 1e-6) / 1e9, 1),
         "quantize_act_gbs": round(qa_bytes / (qa_us * 1e-6) / 1e9, 1),
+        "host_us_per_step": round(host_us, 2),
         "layer_roofline_us": round(layer_roof_us, 2),
         "layer_roofline_frac": round(layer_roof_us / (1e3 * ms_per_step), 4),
         "roofline": {
